@@ -1,1 +1,12 @@
-"""B200-native training RMSNorm (forward, backward, residual form) behind a C-ABI library."""
+"""B200-native training RMSNorm (forward, backward with deterministic or blocked-FP32
+dw, fused residual add, per-head views) behind the C-ABI library librmsnorm_train.
+
+The library is loaded on first use and its absence is an error: there is no CPU or
+eager fallback.
+"""
+
+from .api import (Workspace, bwd_path, det_plan, rmsnorm_train_bwd, rmsnorm_train_fwd,
+                  set_small_rows_limit, status)
+
+__all__ = ["Workspace", "bwd_path", "det_plan", "rmsnorm_train_bwd", "rmsnorm_train_fwd",
+           "set_small_rows_limit", "status"]

@@ -1,0 +1,397 @@
+// C ABI of librmsnorm_train: argument checks, workspace layout, program choice.
+// The declarations and their contract are in include/rmsnorm_train.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "rmsnorm_train.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int ok() {
+    g_err.clear();
+    return RMS_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(RMS_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxH = 8192;
+constexpr int kFoldSegments = 16;
+constexpr size_t kWsHeader = 256;  // status word, ticket
+
+int64_t g_small_rows_override = -1;
+
+struct Span {
+    uintptr_t lo, hi;  // [lo, hi)
+    const char* name;
+};
+
+bool overlap(const Span& a, const Span& b) {
+    return a.lo < a.hi && b.lo < b.hi && a.lo < b.hi && b.lo < a.hi;
+}
+
+int check_shape(const rms_shape& s) {
+    if (s.T < 0) return fail(RMS_EINVAL, "T must be >= 0 (got %lld)", (long long)s.T);
+    if (s.heads < 1) return fail(RMS_EINVAL, "heads must be >= 1 (got %d)", s.heads);
+    if (s.H < 8 || s.H > kMaxH || s.H % 8 != 0)
+        return fail(RMS_EINVAL, "H must be a multiple of 8 in [8, %d] (got %d)", kMaxH, s.H);
+    if (s.T > 0 && (int64_t)s.T * s.heads >= (int64_t(1) << 31))
+        return fail(RMS_EINVAL, "T*heads must be < 2^31");
+    return RMS_OK;
+}
+
+// Checks a row view; appends its byte span.  `out` marks views that are written.
+int check_rows(const rms_shape& s, const rms_rows& v, const char* name, bool out, Span* span) {
+    if (!v.ptr) return fail(RMS_EINVAL, "%s is null", name);
+    if (reinterpret_cast<uintptr_t>(v.ptr) % 16)
+        return fail(RMS_EALIGN, "%s must be 16-byte aligned", name);
+    const int64_t sk = s.heads > 1 ? v.sk : 0;
+    if (v.st < 0 || sk < 0) return fail(RMS_EINVAL, "%s strides must be >= 0", name);
+    if (v.st % 8 || sk % 8)
+        return fail(RMS_EALIGN, "%s strides must be multiples of 8 elements", name);
+    if (out) {
+        if (s.heads > 1 && sk < s.H)
+            return fail(RMS_EINVAL, "%s: head stride %lld makes output rows overlap", name,
+                        (long long)sk);
+        if (s.T > 1 && v.st < (int64_t)(s.heads - 1) * sk + s.H)
+            return fail(RMS_EINVAL, "%s: token stride %lld makes output rows overlap", name,
+                        (long long)v.st);
+    }
+    const int64_t n = (s.T - 1) * v.st + (int64_t)(s.heads - 1) * sk + s.H;
+    span->lo = reinterpret_cast<uintptr_t>(v.ptr);
+    span->hi = span->lo + (uintptr_t)n * 2;
+    span->name = name;
+    return RMS_OK;
+}
+
+int check_aliases(const Span* in, int nin, const Span* out, int nout) {
+    for (int i = 0; i < nout; ++i) {
+        for (int j = 0; j < nin; ++j)
+            if (overlap(out[i], in[j]))
+                return fail(RMS_EALIAS, "output %s overlaps input %s", out[i].name, in[j].name);
+        for (int j = i + 1; j < nout; ++j)
+            if (overlap(out[i], out[j]))
+                return fail(RMS_EALIAS, "output %s overlaps output %s", out[i].name,
+                            out[j].name);
+    }
+    return RMS_OK;
+}
+
+Span span_of(const void* p, size_t bytes, const char* name) {
+    Span s;
+    s.lo = reinterpret_cast<uintptr_t>(p);
+    s.hi = s.lo + bytes;
+    s.name = name;
+    return s;
+}
+
+rmsk::RowsIn in_of(const rms_shape& s, const rms_rows& v) {
+    return {static_cast<const uint16_t*>(v.ptr), v.st, s.heads > 1 ? v.sk : 0};
+}
+rmsk::RowsOut out_of(const rms_shape& s, const rms_rows& v) {
+    return {static_cast<uint16_t*>(v.ptr), v.st, s.heads > 1 ? v.sk : 0};
+}
+
+// ---- the deterministic order and the program choice --------------------------------------
+
+int32_t det_block_rows(int64_t R) {
+    if (R <= 2048) return 16;
+    if (R <= 32768) return 32;
+    return 64;
+}
+
+int64_t default_small_rows(int H) {
+    // single-launch program up to about 2^20 elements (and its shared-memory bound)
+    int64_t lim = (int64_t(1) << 20) / H;
+    if (lim > 2048) lim = 2048;
+    if (lim < 64) lim = 64;
+    return lim;
+}
+
+bool use_small(int64_t R, int H) {
+    const int64_t lim = g_small_rows_override >= 0 ? g_small_rows_override : default_small_rows(H);
+    return R <= lim && R <= 2048;
+}
+
+struct Plan {
+    int32_t B, L, S, n_chunks;
+};
+
+Plan det_plan(int64_t R, int H) {
+    Plan p;
+    p.B = det_block_rows(R);
+    p.L = rmsk::bwd_slots_for_width(H);
+    p.S = kFoldSegments;
+    const int64_t ch = (int64_t)p.B * p.L;
+    p.n_chunks = (int32_t)((R + ch - 1) / ch);
+    return p;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t ws_bytes(const rms_shape& s, int det) {
+    const int64_t R = s.T * s.heads;
+    size_t b = kWsHeader + align256((size_t)s.H * 8);
+    if (det && !use_small(R, s.H)) b += (size_t)det_plan(R, s.H).n_chunks * s.H * 8;
+    return b;
+}
+
+int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const float* rstd,
+               rms_rows dy, const rms_rows* dh, rms_rows dx, float* dw, int deterministic,
+               void* ws, size_t ws_size, int grid_ctas, void* stream) {
+    int rc = check_shape(shape);
+    if (rc) return rc;
+    if (w_dtype != RMS_BF16 && w_dtype != RMS_FP32)
+        return fail(RMS_EDTYPE, "w_dtype must be RMS_BF16 or RMS_FP32 (got %d)", w_dtype);
+    if (grid_ctas < 0 || grid_ctas > 65535)
+        return fail(RMS_EINVAL, "grid_ctas must be in [0, 65535] (got %d)", grid_ctas);
+    if (!w || !dw) return fail(RMS_EINVAL, "w and dw must not be null");
+    if (reinterpret_cast<uintptr_t>(w) % 16 || reinterpret_cast<uintptr_t>(dw) % 16)
+        return fail(RMS_EALIGN, "w and dw must be 16-byte aligned");
+    const int64_t R = shape.T * shape.heads;
+    const int H = shape.H;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t wb = (size_t)H * (w_dtype == RMS_FP32 ? 4 : 2);
+    if (R == 0) {
+        Span ins[1] = {span_of(w, wb, "w")};
+        Span outs[1] = {span_of(dw, (size_t)H * 4, "dw")};
+        if ((rc = check_aliases(ins, 1, outs, 1))) return rc;
+        cudaError_t e = cudaMemsetAsync(dw, 0, (size_t)H * 4, st);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "cudaMemsetAsync(dw)");
+    }
+    if (!rstd) return fail(RMS_EINVAL, "rstd is null");
+    if (reinterpret_cast<uintptr_t>(rstd) % 4) return fail(RMS_EALIGN, "rstd must be 4-byte aligned");
+    Span ins[5], outs[2];
+    int nin = 0;
+    if ((rc = check_rows(shape, x, dh ? "h" : "x", false, &ins[nin++]))) return rc;
+    if ((rc = check_rows(shape, dy, "dy", false, &ins[nin++]))) return rc;
+    if (dh && (rc = check_rows(shape, *dh, "dh", false, &ins[nin++]))) return rc;
+    ins[nin++] = span_of(w, wb, "w");
+    ins[nin++] = span_of(rstd, (size_t)R * 4, "rstd");
+    if ((rc = check_rows(shape, dx, dh ? "grad_h" : "dx", true, &outs[0]))) return rc;
+    outs[1] = span_of(dw, (size_t)H * 4, "dw");
+    if ((rc = check_aliases(ins, nin, outs, 2))) return rc;
+    const size_t need = ws_bytes(shape, deterministic);
+    if (!ws) return fail(RMS_EWORKSPACE, "workspace is null (needs %zu bytes)", need);
+    if (reinterpret_cast<uintptr_t>(ws) % 256)
+        return fail(RMS_EALIGN, "workspace must be 256-byte aligned");
+    if (ws_size < need)
+        return fail(RMS_EWORKSPACE, "workspace has %zu bytes, needs %zu", ws_size, need);
+    {
+        Span wsp = span_of(ws, need, "workspace");
+        for (int i = 0; i < nin; ++i)
+            if (overlap(wsp, ins[i])) return fail(RMS_EALIAS, "workspace overlaps %s", ins[i].name);
+        for (int i = 0; i < 2; ++i)
+            if (overlap(wsp, outs[i])) return fail(RMS_EALIAS, "workspace overlaps %s", outs[i].name);
+    }
+
+    rmsk::BwdParams p = {};
+    p.R = (int32_t)R;
+    p.heads = shape.heads;
+    p.H = H;
+    p.nvec = H / 8;
+    p.x = in_of(shape, x);
+    p.dy = in_of(shape, dy);
+    if (dh) p.dh = in_of(shape, *dh);
+    p.dx = out_of(shape, dx);
+    p.w = w;
+    p.rstd = rstd;
+    p.dw = dw;
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    p.status = reinterpret_cast<unsigned*>(base);
+    p.ticket = reinterpret_cast<unsigned*>(base + 4);
+    p.acc = reinterpret_cast<double*>(base + kWsHeader);
+    p.part = reinterpret_cast<double*>(base + kWsHeader + align256((size_t)H * 8));
+    const Plan plan = det_plan(R, H);
+    p.block_rows = plan.B;
+    p.blocks_per_chunk = plan.L;
+    p.fold_segments = plan.S;
+    p.n_chunks = plan.n_chunks;
+    const bool res = dh != nullptr;
+    const bool w32 = w_dtype == RMS_FP32;
+    cudaError_t e;
+    if (use_small(R, H)) {
+        e = rmsk::launch_bwd_small(p, res, w32, st);
+    } else if (deterministic) {
+        e = rmsk::launch_bwd_det(p, res, w32, grid_ctas, st);
+    } else {
+        e = rmsk::launch_bwd_nondet(p, res, w32, grid_ctas, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    return ok();
+}
+
+}  // namespace
+
+namespace rmsk {
+
+int device_sm_count() {
+    static int cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+}  // namespace rmsk
+
+extern "C" {
+
+int rms_train_fwd(rms_shape shape, rms_rows x, const void* w, int w_dtype, rms_rows y,
+                  float* rstd, float eps, void* stream) {
+    int rc = check_shape(shape);
+    if (rc) return rc;
+    if (w_dtype != RMS_BF16 && w_dtype != RMS_FP32)
+        return fail(RMS_EDTYPE, "w_dtype must be RMS_BF16 or RMS_FP32 (got %d)", w_dtype);
+    const int64_t R = shape.T * shape.heads;
+    if (R == 0) return ok();
+    if (!w || !rstd) return fail(RMS_EINVAL, "w and rstd must not be null");
+    if (reinterpret_cast<uintptr_t>(w) % 16) return fail(RMS_EALIGN, "w must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(rstd) % 4) return fail(RMS_EALIGN, "rstd must be 4-byte aligned");
+    Span ins[2], outs[2];
+    if ((rc = check_rows(shape, x, "x", false, &ins[0]))) return rc;
+    ins[1] = span_of(w, (size_t)shape.H * (w_dtype == RMS_FP32 ? 4 : 2), "w");
+    if ((rc = check_rows(shape, y, "y", true, &outs[0]))) return rc;
+    outs[1] = span_of(rstd, (size_t)R * 4, "rstd");
+    if ((rc = check_aliases(ins, 2, outs, 2))) return rc;
+    rmsk::FwdParams p = {};
+    p.R = (int32_t)R;
+    p.heads = shape.heads;
+    p.H = shape.H;
+    p.nvec = shape.H / 8;
+    p.x = in_of(shape, x);
+    p.y = out_of(shape, y);
+    p.w = w;
+    p.rstd = rstd;
+    p.eps = eps;
+    cudaError_t e = rmsk::launch_fwd(p, false, w_dtype == RMS_FP32, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "forward launch");
+}
+
+int rms_residual_train_fwd(rms_shape shape, rms_rows x, rms_rows residual, const void* w,
+                           int w_dtype, rms_rows h_out, rms_rows y, float* rstd, float eps,
+                           void* stream) {
+    int rc = check_shape(shape);
+    if (rc) return rc;
+    if (w_dtype != RMS_BF16 && w_dtype != RMS_FP32)
+        return fail(RMS_EDTYPE, "w_dtype must be RMS_BF16 or RMS_FP32 (got %d)", w_dtype);
+    const int64_t R = shape.T * shape.heads;
+    if (R == 0) return ok();
+    if (!w || !rstd) return fail(RMS_EINVAL, "w and rstd must not be null");
+    if (reinterpret_cast<uintptr_t>(w) % 16) return fail(RMS_EALIGN, "w must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(rstd) % 4) return fail(RMS_EALIGN, "rstd must be 4-byte aligned");
+    Span ins[3], outs[3];
+    if ((rc = check_rows(shape, x, "x", false, &ins[0]))) return rc;
+    if ((rc = check_rows(shape, residual, "residual", false, &ins[1]))) return rc;
+    ins[2] = span_of(w, (size_t)shape.H * (w_dtype == RMS_FP32 ? 4 : 2), "w");
+    if ((rc = check_rows(shape, h_out, "h_out", true, &outs[0]))) return rc;
+    if ((rc = check_rows(shape, y, "y", true, &outs[1]))) return rc;
+    outs[2] = span_of(rstd, (size_t)R * 4, "rstd");
+    if ((rc = check_aliases(ins, 3, outs, 3))) return rc;
+    rmsk::FwdParams p = {};
+    p.R = (int32_t)R;
+    p.heads = shape.heads;
+    p.H = shape.H;
+    p.nvec = shape.H / 8;
+    p.x = in_of(shape, x);
+    p.res = in_of(shape, residual);
+    p.h = out_of(shape, h_out);
+    p.y = out_of(shape, y);
+    p.w = w;
+    p.rstd = rstd;
+    p.eps = eps;
+    cudaError_t e = rmsk::launch_fwd(p, true, w_dtype == RMS_FP32, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ok() : cuda_fail(e, "residual forward launch");
+}
+
+int rms_train_bwd(rms_shape shape, rms_rows x, const void* w, int w_dtype, const float* rstd,
+                  rms_rows dy, rms_rows dx, float* dw, int deterministic, void* workspace,
+                  size_t workspace_bytes, int grid_ctas, void* stream) {
+    return bwd_common(shape, x, w, w_dtype, rstd, dy, nullptr, dx, dw, deterministic, workspace,
+                      workspace_bytes, grid_ctas, stream);
+}
+
+int rms_residual_train_bwd(rms_shape shape, rms_rows h, const void* w, int w_dtype,
+                           const float* rstd, rms_rows dy, rms_rows dh, rms_rows grad_h,
+                           float* dw, int deterministic, void* workspace,
+                           size_t workspace_bytes, int grid_ctas, void* stream) {
+    return bwd_common(shape, h, w, w_dtype, rstd, dy, &dh, grad_h, dw, deterministic, workspace,
+                      workspace_bytes, grid_ctas, stream);
+}
+
+size_t rms_train_bwd_workspace_bytes(rms_shape shape, int deterministic, int grid_ctas) {
+    (void)grid_ctas;  // the layout does not depend on the grid
+    if (check_shape(shape)) return 0;
+    return ws_bytes(shape, deterministic);
+}
+
+int rms_det_plan(rms_shape shape, int32_t* block_rows, int32_t* blocks_per_chunk,
+                 int32_t* fold_segments) {
+    int rc = check_shape(shape);
+    if (rc) return rc;
+    const Plan p = det_plan(shape.T * shape.heads, shape.H);
+    if (block_rows) *block_rows = p.B;
+    if (blocks_per_chunk) *blocks_per_chunk = p.L;
+    if (fold_segments) *fold_segments = p.S;
+    return ok();
+}
+
+int rms_train_bwd_path(rms_shape shape, int deterministic) {
+    int rc = check_shape(shape);
+    if (rc) return rc;
+    const int64_t R = shape.T * shape.heads;
+    if (use_small(R, shape.H)) return 1;
+    return deterministic ? 2 : 3;
+}
+
+int64_t rms_set_small_rows_limit(int64_t rows) {
+    const int64_t prev = g_small_rows_override;
+    g_small_rows_override = rows < 0 ? -1 : rows;
+    return prev;
+}
+
+int rms_status(void* workspace, void* stream) {
+    if (!workspace) return fail(RMS_EINVAL, "workspace is null");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned word = 0;
+    e = cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+    if (word) {
+        e = cudaMemset(workspace, 0, sizeof word);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status)");
+        if (word & rmsk::kStatusTimeout)
+            return fail(RMS_ETIMEOUT, "a device-side bounded wait gave up (status 0x%x)", word);
+        return fail(RMS_ECUDA, "device status 0x%x", word);
+    }
+    return ok();
+}
+
+const char* rms_last_error(void) { return g_err.c_str(); }
+
+int rms_device_sms(void) { return rmsk::device_sm_count(); }
+
+}  // extern "C"

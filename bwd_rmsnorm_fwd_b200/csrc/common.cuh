@@ -1,0 +1,169 @@
+// Internal declarations shared by the kernels and the C-ABI layer of librmsnorm_train.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rmsk {
+
+// A [T, heads, H] row view: row (t, k) starts at element t*st + k*sk.
+struct RowsIn {
+    const uint16_t* ptr;
+    int64_t st, sk;
+};
+struct RowsOut {
+    uint16_t* ptr;
+    int64_t st, sk;
+};
+
+struct FwdParams {
+    int32_t R;       // rows = T * heads
+    int32_t heads;
+    int32_t H;
+    int32_t nvec;    // H / 8 (16-byte vectors per row)
+    RowsIn x;
+    RowsIn res;      // residual form only
+    RowsOut h;       // residual form only
+    RowsOut y;
+    const void* w;
+    float* rstd;
+    float eps;
+};
+
+struct BwdParams {
+    int32_t R;
+    int32_t heads;
+    int32_t H;
+    int32_t nvec;
+    RowsIn x;        // h in the residual form
+    RowsIn dy;
+    RowsIn dh;       // residual form only
+    RowsOut dx;      // grad_h in the residual form
+    const void* w;
+    const float* rstd;
+    float* dw;
+    // workspace pieces
+    unsigned* status;    // device error word
+    unsigned* ticket;    // non-deterministic grid combine
+    double* acc;         // [H] FP64, zero between calls
+    double* part;        // [n_chunks, H] FP64 chunk partials (deterministic)
+    // deterministic order
+    int32_t block_rows;
+    int32_t blocks_per_chunk;
+    int32_t fold_segments;
+    int32_t n_chunks;
+};
+
+// device status bits
+constexpr unsigned kStatusTimeout = 1u;
+
+// ---- host-side launchers (defined in fwd.cu / bwd.cu) -------------------------------------
+
+cudaError_t launch_fwd(const FwdParams& p, bool residual, bool w32, cudaStream_t s);
+cudaError_t launch_bwd_small(const BwdParams& p, bool residual, bool w32, cudaStream_t s);
+cudaError_t launch_bwd_det(const BwdParams& p, bool residual, bool w32, int grid_ctas,
+                           cudaStream_t s);
+cudaError_t launch_bwd_nondet(const BwdParams& p, bool residual, bool w32, int grid_ctas,
+                              cudaStream_t s);
+
+// Rows processed together by one CTA of the large backward kernels for this width
+// (the blocks of one deterministic chunk).  Also the chunk's block count.
+int bwd_slots_for_width(int H);
+int device_sm_count();
+
+}  // namespace rmsk
+
+// ---- device helpers ------------------------------------------------------------------------
+#ifdef __CUDACC__
+namespace rmsk {
+
+__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// two FP32 -> packed BF16x2, round to nearest even (low half = a)
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x);
+    f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z);
+    f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+    uint4 v;
+    v.x = pack_bf16x2(f[0], f[1]);
+    v.y = pack_bf16x2(f[2], f[3]);
+    v.z = pack_bf16x2(f[4], f[5]);
+    v.w = pack_bf16x2(f[6], f[7]);
+    return v;
+}
+
+// 16-byte streaming load of data read once (no L1 allocation).
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(p));
+    return v;
+}
+
+// 16-byte load through L1 (small, reused data: the weight).
+__device__ __forceinline__ uint4 ld_cached16(const void* p) {
+    return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ void st16(void* p, const uint4& v) {
+    *reinterpret_cast<uint4*>(p) = v;
+}
+
+// 8 weights as FP32 from a BF16 or FP32 weight vector, element offset e (multiple of 8).
+template <bool W32>
+__device__ __forceinline__ void load_w8(const void* w, int e, float (&f)[8]) {
+    if constexpr (W32) {
+        const float* wf = static_cast<const float*>(w) + e;
+        uint4 a = ld_cached16(wf), b = ld_cached16(wf + 4);
+        f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y);
+        f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
+        f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y);
+        f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+    } else {
+        uint4 a = ld_cached16(static_cast<const uint16_t*>(w) + e);
+        unpack8(a, f);
+    }
+}
+
+__device__ __forceinline__ int64_t row_offset(int32_t r, int32_t heads, int64_t st,
+                                              int64_t sk) {
+    if (heads == 1) return (int64_t)r * st;
+    const int32_t t = r / heads;
+    const int32_t k = r - t * heads;
+    return (int64_t)t * st + (int64_t)k * sk;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+// TwoSum accumulation of the exact product a*b into (s, c):  p + e == a*b exactly,
+// t + err == s + p exactly; the rounding errors go to the compensation term c.
+// Written with explicit round-to-nearest intrinsics so nothing is contracted or
+// reassociated: the deterministic order depends on this exact sequence.
+__device__ __forceinline__ void twosum_product(float a, float b, float& s, float& c) {
+    const float p = __fmul_rn(a, b);
+    const float e = __fmaf_rn(a, b, -p);
+    const float t = __fadd_rn(s, p);
+    const float z = __fsub_rn(t, s);
+    const float err = __fadd_rn(__fsub_rn(s, __fsub_rn(t, z)), __fsub_rn(p, z));
+    c = __fadd_rn(c, __fadd_rn(err, e));
+    s = t;
+}
+
+}  // namespace rmsk
+#endif

@@ -1,0 +1,155 @@
+/*
+ * librmsnorm_train -- training RMSNorm for NVIDIA B200 (sm_100a), C ABI.
+ *
+ * The operation (flashinfer PR #8848 "...sm_100a non-deterministic backward...",
+ * introduction and "Measurement"/"Workload"; flashinfer PR #8512 "fix(cake_rmsnorm_det):
+ * fixed-order dw for the smallest token counts of the SM100/SM103 backward", introduction):
+ *
+ *   forward   rstd_r = 1 / sqrt(mean_j(x_rj^2) + eps)          FP32 [R]
+ *             y_rj   = x_rj * rstd_r * w_j                      BF16, x's layout
+ *   backward  xh = x * rstd, g = dy * w, c_r = (1/H) sum_j g_rj xh_rj
+ *             dx_rj  = rstd_r * (g_rj - xh_rj * c_r)            BF16
+ *             dw_j   = sum_r dy_rj * xh_rj                      FP32 [H]
+ *   residual  h = BF16(x + residual) and the forward runs on h (h is returned);
+ *             the backward takes dy and dh and returns grad_h = BF16(dh + dx)
+ *             (PR #8512 introduction, "Residual rows"; PR #8848 "Key").
+ *
+ * Two backward modes (PR #8512 introduction; PR #8848 introduction):
+ *   deterministic != 0  every dw column is summed over a fixed row order with exact
+ *                       products and TwoSum compensation, the pieces are folded in a
+ *                       fixed FP64 order and rounded once to FP32.  The order depends
+ *                       only on (rows, H) -- never on grid_ctas or the SM count -- so dw
+ *                       is bit-identical across grids; rms_det_plan() returns it.
+ *   deterministic == 0  blocked FP32 sums (eight rows per block) per thread, combined
+ *                       in FP64 across the grid in arrival order.
+ *
+ * Layout.  A row tensor is a [T, heads, H] view: row (t, k) starts at element
+ * ptr + t*st + k*sk and its H elements are contiguous.  Rows are numbered
+ * r = t*heads + k (R = T*heads); rstd is a dense FP32 [R] array in that order.
+ * Per-head views such as [T,24,256] with strides (12288, 512, 1) or dense
+ * [T,4,256] share one w[H] (PR #8848 introduction; PR #8512 squashed commit of #8626).
+ * x/y/dy/dx/h/residual/dh/grad_h are BF16; w is BF16 or FP32; dw is FP32.
+ *
+ * Requirements (checked on the host before anything is launched; a failing call
+ * writes nothing):  1 <= H <= 8192, H % 8 == 0; heads >= 1; T >= 0; T*heads < 2^31;
+ * every row pointer, w and dw 16-byte aligned; st and sk multiples of 8 elements;
+ * rstd 4-byte aligned; no output range overlaps an input range or another output
+ * (dw aliasing w is rejected, PR #8512 review "Reject dw that aliases w").
+ *
+ * Ownership.  The caller owns every buffer, the workspace included.  The library
+ * allocates no device memory, never synchronises inside the compute calls, and
+ * launches only 1-D grids (PR #8848 review "Reject non-one-dimensional grids").
+ * All calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *
+ * Errors.  Every entry point returns RMS_OK or a negative code; rms_last_error()
+ * gives a message (thread-local).  Launch failures return RMS_ECUDA.  Conditions the
+ * device detects are written to the workspace status word; rms_status() reads them.
+ */
+#ifndef RMSNORM_TRAIN_H
+#define RMSNORM_TRAIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types: BF16 (bfloat16 bits) or FP32. */
+enum { RMS_BF16 = 0, RMS_FP32 = 1 };
+
+/* Return codes. */
+enum {
+    RMS_OK = 0,
+    RMS_EINVAL = -1,     /* bad shape, null pointer, bad stride, bad grid_ctas   */
+    RMS_EDTYPE = -2,     /* unsupported dtype code                                 */
+    RMS_EALIGN = -3,     /* pointer or stride not aligned as required               */
+    RMS_EALIAS = -4,     /* an output overlaps an input or another output           */
+    RMS_EWORKSPACE = -5, /* workspace missing or smaller than the size query says   */
+    RMS_ECUDA = -6,      /* a CUDA runtime call or launch failed                    */
+    RMS_ETIMEOUT = -7    /* a device-side bounded wait gave up (rms_status)         */
+};
+
+/* A [T, heads, H] row view; strides in elements, innermost stride 1. */
+typedef struct {
+    void* ptr;
+    int64_t st; /* stride between tokens t   */
+    int64_t sk; /* stride between heads k    */
+} rms_rows;
+
+typedef struct {
+    int64_t T;     /* tokens (rows per head) */
+    int32_t heads; /* rows per token         */
+    int32_t H;     /* row width              */
+} rms_shape;
+
+/* Forward.  Reads x [T,heads,H] BF16 and w [H] (w_dtype), writes y (BF16, its own
+ * strides) and rstd (FP32 [R]).  eps is added to the mean of squares (1e-6 on the
+ * pages, PR #8848 "Workload").  T == 0 is a no-op. */
+int rms_train_fwd(rms_shape shape, rms_rows x, const void* w, int w_dtype, rms_rows y,
+                  float* rstd, float eps, void* stream);
+
+/* Residual forward.  h_out = BF16(x + residual); then the forward of rms_train_fwd on
+ * h_out.  Writes h_out, y and rstd. */
+int rms_residual_train_fwd(rms_shape shape, rms_rows x, rms_rows residual, const void* w,
+                           int w_dtype, rms_rows h_out, rms_rows y, float* rstd, float eps,
+                           void* stream);
+
+/* Backward.  Reads x (the forward's input), w, rstd (the forward's FP32 output) and dy;
+ * writes dx (BF16) and dw (FP32 [H], overwritten, not accumulated).  The workspace
+ * (>= rms_train_bwd_workspace_bytes(shape, deterministic, grid_ctas) bytes, 256-byte
+ * aligned) must be zero-filled once before its first use; every call leaves it ready
+ * for the next.  Calls sharing a workspace must be stream-ordered.  grid_ctas = 0 picks
+ * the grid; any other value (1 .. 65535) sets the CTA count of the main backward kernel
+ * and never changes the deterministic dw bits.  T == 0 writes dw = 0. */
+int rms_train_bwd(rms_shape shape, rms_rows x, const void* w, int w_dtype, const float* rstd,
+                  rms_rows dy, rms_rows dx, float* dw, int deterministic, void* workspace,
+                  size_t workspace_bytes, int grid_ctas, void* stream);
+
+/* Residual backward.  h is the forward's h_out; dy the gradient of y, dh the gradient of
+ * h.  Writes grad_h = BF16(dh + dx) and dw.  Workspace rules as rms_train_bwd. */
+int rms_residual_train_bwd(rms_shape shape, rms_rows h, const void* w, int w_dtype,
+                           const float* rstd, rms_rows dy, rms_rows dh, rms_rows grad_h,
+                           float* dw, int deterministic, void* workspace,
+                           size_t workspace_bytes, int grid_ctas, void* stream);
+
+/* Workspace bytes the backward needs for this shape, mode and grid (0 on bad input). */
+size_t rms_train_bwd_workspace_bytes(rms_shape shape, int deterministic, int grid_ctas);
+
+/* The fixed deterministic summation order for this shape: rows are cut into blocks of
+ * *block_rows; each block is summed in row order with exact products and TwoSum and
+ * converted to FP64 (sum + compensation); *blocks_per_chunk consecutive blocks are
+ * folded left to right in FP64 into one chunk partial; the chunk partials are cut into
+ * *fold_segments contiguous segments of ceil(chunks / segments) chunks, each folded left
+ * to right, and the segment sums are folded left to right and rounded once to FP32.
+ * Returns RMS_OK or RMS_EINVAL. */
+int rms_det_plan(rms_shape shape, int32_t* block_rows, int32_t* blocks_per_chunk,
+                 int32_t* fold_segments);
+
+/* Which backward program a call with this shape runs: 1 = single-launch small-row
+ * kernel (row tasks + column tasks), 2 = main kernel + fixed-order fold kernel
+ * (deterministic), 3 = single kernel with FP64 grid combine (non-deterministic).
+ * Negative on bad input. */
+int rms_train_bwd_path(rms_shape shape, int deterministic);
+
+/* Largest row count R (= T*heads) served by the single-launch small-row program; the
+ * default is chosen from H.  Setting a value >= 0 overrides it for every later call
+ * in this process (not thread-safe against concurrent backward calls); -1 restores
+ * the default.  Returns the previous override (-1 if none). */
+int64_t rms_set_small_rows_limit(int64_t rows);
+
+/* Synchronises `stream`, reads and clears the device status word of `workspace`.
+ * Returns RMS_OK, RMS_ETIMEOUT or RMS_ECUDA. */
+int rms_status(void* workspace, void* stream);
+
+/* Message for the last non-zero return on this thread ("" if none). */
+const char* rms_last_error(void);
+
+/* Number of SMs of the current device (0 on error). */
+int rms_device_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RMSNORM_TRAIN_H */

@@ -1,0 +1,131 @@
+"""Deterministic dw: bit-identical across grids, repeats and programs, and equal bit for
+bit to a CPU emulation of the documented summation order (a test of the order, kept
+apart from the FP64 oracle, which defines the value)."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bwd_rmsnorm_fwd_b200 import api, synth
+
+from gpu_common import dev_rows, dev_weight
+
+pytestmark = pytest.mark.gpu
+
+
+def emulate_det_dw(x_bits, dy_bits, rstd, B, L, S):
+    """IEEE emulation of the fixed order: per column, blocks of B rows summed in row order
+    with exact products (p + e == dy * xh) and TwoSum; each block -> FP64 (s + c); L blocks
+    per chunk folded left to right; S contiguous segments of chunks folded left to right;
+    the segment sums folded left to right; one rounding to FP32."""
+    x = synth.bf16_bits_to_f32(x_bits)
+    dy = synth.bf16_bits_to_f32(dy_bits)
+    R, H = x.shape
+    rstd = rstd.astype(np.float32)
+    n_blocks = -(-R // B)
+    bp = np.empty((n_blocks, H), np.float64)
+    for b in range(n_blocks):
+        s = np.zeros(H, np.float32)
+        c = np.zeros(H, np.float32)
+        for r in range(b * B, min(R, (b + 1) * B)):
+            xh = x[r] * rstd[r]                                   # FP32, nearest
+            p = dy[r] * xh
+            e = (dy[r].astype(np.float64) * xh.astype(np.float64) - p).astype(np.float32)
+            t = s + p
+            z = t - s
+            err = (s - (t - z)) + (p - z)
+            c = c + (err + e)
+            s = t
+        bp[b] = s.astype(np.float64) + c.astype(np.float64)
+    n_chunks = -(-n_blocks // L)
+    chunks = []
+    for k in range(n_chunks):
+        a = bp[k * L].copy()
+        for b in range(k * L + 1, min(n_blocks, (k + 1) * L)):
+            a = a + bp[b]
+        chunks.append(a)
+    seg_len = -(-n_chunks // S)
+    total = None
+    for q in range(S):
+        k0, k1 = q * seg_len, min(n_chunks, (q + 1) * seg_len)
+        if k0 >= k1:
+            continue
+        sg = chunks[k0].copy()
+        for k in range(k0 + 1, k1):
+            sg = sg + chunks[k]
+        total = sg if total is None else total + sg
+    return total.astype(np.float32)
+
+
+def inputs(T, heads, H, seed=0, family="F1", wdt="bf16"):
+    R = T * heads
+    x = synth.rows(seed, "x", R, H, family)
+    dy = synth.rows(seed, "dy", R, H, family)
+    w = synth.weight(seed, H, wdt)
+    _, rstd = oracle.train_fwd(x, w)
+    return x, dy, w, rstd
+
+
+def gpu_dw(x, dy, w, rstd, det=True, grid=0, heads=1, res_dh=None):
+    H = x.shape[1]
+    xd = dev_rows(x).reshape(-1, heads, H) if heads > 1 else dev_rows(x)
+    dyd = dev_rows(dy).reshape(xd.shape)
+    dh = None if res_dh is None else dev_rows(res_dh).reshape(xd.shape)
+    _, dw = api.rmsnorm_train_bwd(xd, dev_weight(w), torch.from_numpy(rstd).cuda(), dyd,
+                                  deterministic=det, grid_ctas=grid, dh=dh)
+    torch.cuda.synchronize()
+    return dw.cpu().numpy()
+
+
+@pytest.mark.parametrize("T,heads,H", [(70001, 1, 6144), (9000, 1, 1536), (4096, 24, 256),
+                                       (20000, 1, 4096), (50000, 1, 2048), (30000, 4, 256)])
+def test_bits_identical_across_grids_and_repeats(T, heads, H):
+    x, dy, w, rstd = inputs(T, heads, H, seed=5, family="F3")
+    ref = gpu_dw(x, dy, w, rstd, heads=heads)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for grid in (1, 7, 37, sms, 2 * sms, 3 * sms + 1, 1000):
+        got = gpu_dw(x, dy, w, rstd, grid=grid, heads=heads)
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), grid
+    for _ in range(3):
+        assert np.array_equal(gpu_dw(x, dy, w, rstd, heads=heads).view(np.uint32),
+                              ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("T,H", [(227, 4096), (1000, 512), (2048, 256), (600, 1536)])
+def test_single_launch_and_pair_give_the_same_bits(T, H):
+    x, dy, w, rstd = inputs(T, 1, H, seed=6, family="F2")
+    prev = api.set_small_rows_limit(1 << 30)
+    try:
+        assert api.bwd_path(T, 1, H, True) == 1
+        a = gpu_dw(x, dy, w, rstd)
+        api.set_small_rows_limit(0)
+        assert api.bwd_path(T, 1, H, True) == 2
+        b = gpu_dw(x, dy, w, rstd)
+        c = gpu_dw(x, dy, w, rstd, grid=3)
+    finally:
+        api.set_small_rows_limit(prev)
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    assert np.array_equal(a.view(np.uint32), c.view(np.uint32))
+
+
+@pytest.mark.parametrize("T,heads,H", [(227, 1, 512), (5000, 1, 1536), (4100, 1, 6144),
+                                       (700, 24, 256), (33000, 1, 264)])
+def test_bits_equal_cpu_emulation_of_the_order(T, heads, H):
+    x, dy, w, rstd = inputs(T, heads, H, seed=7, family="F3", wdt="fp32")
+    B, L, S = api.det_plan(T, heads, H)
+    want = emulate_det_dw(x, dy, rstd, B, L, S)
+    got = gpu_dw(x, dy, w, rstd, heads=heads)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+def test_residual_form_bits_do_not_depend_on_grid():
+    T, H = 5000, 6144
+    x, dy, w, rstd = inputs(T, 1, H, seed=8)
+    dh = synth.rows(8, "dh", T, H)
+    ref = gpu_dw(x, dy, w, rstd, res_dh=dh)
+    for grid in (5, 148, 999):
+        assert np.array_equal(gpu_dw(x, dy, w, rstd, grid=grid, res_dh=dh).view(np.uint32),
+                              ref.view(np.uint32))

@@ -1,0 +1,196 @@
+"""GPU vs oracle parity, element by element, on seeded inputs shaped like the pages'
+workloads.  Every call goes through the C ABI (via the thin torch binding)."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bwd_rmsnorm_fwd_b200 import api, synth
+
+from gpu_common import (assert_dw, assert_dx, assert_fwd, bf16_ulps, dev_rows, dev_weight,
+                        dw_ratio, empty_strided_buffer, f32, gaps_untouched, host_bits,
+                        strided_buffer, view_rows)
+
+pytestmark = pytest.mark.gpu
+
+EPS = 1e-6
+
+
+def run_case(T, heads, H, wdt, seed=0, family="F1", residual=False, modes=(True, False),
+             layout=None, grid_ctas=0):
+    """Full-oracle parity of the forward and both backward modes on one shape.
+    layout = (st, sk) strides for a per-head view (default: dense)."""
+    R = T * heads
+    st, sk = layout if layout else (heads * H, H)
+    x = synth.rows(seed, "x", R, H, family)
+    dy = synth.rows(seed, "dy", R, H, family)
+    w = synth.weight(seed, H, wdt)
+    wd = dev_weight(w)
+    xbuf, xv = strided_buffer(x, T, heads, H, st, sk)
+    dybuf, dyv = strided_buffer(dy, T, heads, H, st, sk)
+    ybuf, yv = empty_strided_buffer(T, heads, H, st, sk)
+    if residual:
+        res = synth.rows(seed, "res", R, H, family)
+        dh = synth.rows(seed, "dh", R, H, family)
+        rbuf, rv = strided_buffer(res, T, heads, H, st, sk)
+        dhbuf, dhv = strided_buffer(dh, T, heads, H, st, sk)
+        hbuf, hv = empty_strided_buffer(T, heads, H, st, sk)
+        h_ref, y_ref, rstd_ref = oracle.train_fwd(x, w, EPS, residual=res)
+        _, _, rstd = api.rmsnorm_train_fwd(xv, wd, EPS, residual=rv, y=yv, h_out=hv)
+        assert np.array_equal(view_rows(hv), h_ref), "h is not bit-exact"
+        assert gaps_untouched(hbuf, T, heads, H, st, sk)
+        xin, xin_v = h_ref, hv
+    else:
+        y_ref, rstd_ref = oracle.train_fwd(x, w, EPS)
+        _, rstd = api.rmsnorm_train_fwd(xv, wd, EPS, y=yv)
+        dh = dhv = None
+        xin, xin_v = x, xv
+    torch.cuda.synchronize()
+    assert_fwd(view_rows(yv), rstd.cpu().numpy(), y_ref, rstd_ref, f"fwd {T}x{heads}x{H}")
+    assert gaps_untouched(ybuf, T, heads, H, st, sk)
+    # both backwards take the oracle's FP32 rstd: no oracle input comes from the GPU
+    dx_ref, dw_ref = oracle.train_bwd(xin, w, rstd_ref, dy, dh=dh)
+    rstd_in = torch.from_numpy(rstd_ref).cuda()
+    out = {}
+    for det in modes:
+        dxbuf, dxv = empty_strided_buffer(T, heads, H, st, sk)
+        _, dw = api.rmsnorm_train_bwd(xin_v, wd, rstd_in, dyv, deterministic=det, dh=dhv,
+                                      dx=dxv, grid_ctas=grid_ctas)
+        api.status()
+        torch.cuda.synchronize()
+        assert_dx(view_rows(dxv), dx_ref, f"dx det={det}")
+        assert gaps_untouched(dxbuf, T, heads, H, st, sk)
+        dwh = dw.cpu().numpy()
+        if det or family == "F1":
+            assert_dw(dwh, dw_ref, f"dw det={det} {T}x{heads}x{H} {wdt} {family}")
+        out[det] = dwh
+    return out, dw_ref
+
+
+# ---- BASELINE configurations -----------------------------------------------------------
+
+def test_tiny_config():
+    """T=64, H=512, x BF16 N(0,1), FP32 weight 1+0.1N(0,1), dy N(0,1), eps 1e-6; fwd then
+    deterministic bwd, seed 0."""
+    run_case(64, 1, 512, "fp32", seed=0)
+
+
+@pytest.mark.parametrize("wdt", ["bf16", "fp32"])
+@pytest.mark.parametrize("T", [1, 2, 8, 32, 87, 227])
+@pytest.mark.parametrize("H", [256, 512, 2048, 4096])
+def test_small_t_sweep(H, T, wdt):
+    out, _ = run_case(T, 1, H, wdt, seed=T + H)
+    # both modes run the single-launch program here: identical bits
+    assert np.array_equal(out[True], out[False])
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_small_t_worst_of_five_seeds(seed):
+    for H, T in [(512, 227), (4096, 87), (256, 32)]:
+        run_case(T, 1, H, "bf16", seed=seed, modes=(True,))
+
+
+@pytest.mark.parametrize("T", [32, 4096, 65537])
+def test_residual_h6144(T):
+    run_case(T, 1, 6144, "bf16", seed=1, residual=True)
+
+
+@pytest.mark.parametrize("wdt", ["fp32", "bf16"])
+@pytest.mark.parametrize("T", [1024, 16384])
+@pytest.mark.parametrize("view", ["24x256_pages", "24x256_dense", "4x256"])
+def test_per_head_views(view, T, wdt):
+    heads, layout = {"24x256_pages": (24, (12288, 512)), "24x256_dense": (24, (6144, 256)),
+                     "4x256": (4, (1024, 256))}[view]
+    run_case(T, heads, 256, wdt, seed=2, layout=layout)
+
+
+@pytest.mark.parametrize("wdt", ["bf16", "fp32"])
+@pytest.mark.parametrize("H", [1536, 2048, 4096, 5120, 6144])
+def test_large_widths_ragged_rows(H, wdt):
+    """Every large-T width at a row count that spans many chunks and ends in a ragged tail."""
+    run_case(4099, 1, H, wdt, seed=H)
+
+
+# ---- edge cases ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("H", [8, 24, 264, 776, 8192])
+def test_ragged_and_extreme_widths(H):
+    for T in (1, 3, 3001):
+        run_case(T, 1, H, "fp32", seed=H + T)
+
+
+def test_zero_rows():
+    w = dev_weight(synth.weight(0, 512, "fp32"))
+    x = torch.empty(0, 512, dtype=torch.bfloat16, device="cuda")
+    y, rstd = api.rmsnorm_train_fwd(x, w)
+    dw = torch.full((512,), 7.0, device="cuda")
+    dx, dw = api.rmsnorm_train_bwd(x, w, rstd, x, dw=dw)
+    torch.cuda.synchronize()
+    assert y.numel() == 0 and torch.all(dw == 0)
+
+
+def test_cancellation_example_on_gpu():
+    """The pages' review example (65536, 2^-10, -65536 in row order): the deterministic mode
+    returns 2^-10 exactly (the oracle's exact value); the blocked-FP32 mode may lose it when
+    the three rows fall into one eight-row block, which is the documented hazard."""
+    H = 64
+    prods = [65536.0, 2.0 ** -10, -65536.0]
+    x = synth.f32_to_bf16_bits(np.ones((3, H), np.float32))
+    dy = synth.f32_to_bf16_bits(np.repeat(np.array(prods, np.float32)[:, None], H, 1))
+    w = dev_weight(synth.weight(0, H, "fp32"))
+    rstd = torch.ones(3, device="cuda")
+    for path_limit in (-1, 0):  # single-launch program, then the main + fold pair
+        prev = api.set_small_rows_limit(path_limit)
+        try:
+            _, dw = api.rmsnorm_train_bwd(dev_rows(x), w, rstd, dev_rows(dy), deterministic=True)
+            assert torch.all(dw == 2.0 ** -10), dw[:4]
+            _, dwn = api.rmsnorm_train_bwd(dev_rows(x), w, rstd, dev_rows(dy), deterministic=False)
+            vals = set(dwn.cpu().numpy().tolist())
+            assert vals <= {0.0, 2.0 ** -10}
+        finally:
+            api.set_small_rows_limit(prev)
+
+
+@pytest.mark.parametrize("family", ["F1", "F2", "F3"])
+def test_input_families(family):
+    """Deterministic dw meets the budget on all three families; the blocked-FP32 mode is
+    held to it on F1 (asserted in run_case) and its F2/F3 ratios are reported."""
+    for H, T in [(4096, 8192), (256, 40000)]:
+        out, ref = run_case(T, 1, H, "bf16", seed=3, family=family, modes=(True, False))
+        print(f"{family} H{H} T{T}: dw err/tol det {dw_ratio(out[True], ref):.3g} "
+              f"non-det {dw_ratio(out[False], ref):.3g}")
+
+
+def test_fp32_weight_dw_not_worse_than_fp32_eager():
+    """With FP32 weight the pages bound dw error by that of FP32 eager on the same inputs."""
+    T, H = 16384, 2048
+    x = synth.rows(4, "x", T, H)
+    dy = synth.rows(4, "dy", T, H)
+    w = synth.weight(4, H, "fp32")
+    _, rstd_ref = oracle.train_fwd(x, w)
+    _, dw_ref = oracle.train_bwd(x, w, rstd_ref, dy, want_dx=False)
+    xd, dyd, rstd = dev_rows(x), dev_rows(dy), torch.from_numpy(rstd_ref).cuda()
+    eager = (dyd.float() * (xd.float() * rstd[:, None])).sum(0).cpu().numpy()
+    e_eager = np.abs(eager.astype(np.float64) - dw_ref).max()
+    for det in (True, False):
+        _, dw = api.rmsnorm_train_bwd(xd, dev_weight(w), rstd, dyd, deterministic=det)
+        e = np.abs(dw.cpu().numpy().astype(np.float64) - dw_ref).max()
+        assert e <= e_eager, (det, e, e_eager)
+
+
+def test_alias_and_dtype_errors_with_device_tensors():
+    from bwd_rmsnorm_fwd_b200._lib import RmsError, RMS_EALIAS
+    H = 256
+    x = dev_rows(synth.rows(0, "x", 64, H))
+    w = torch.ones(H, device="cuda")
+    y, rstd = api.rmsnorm_train_fwd(x, w)
+    with pytest.raises(RmsError) as ei:
+        api.rmsnorm_train_bwd(x, w, rstd, x.clone(), dw=w)   # dw aliasing w
+    assert ei.value.code == RMS_EALIAS
+    with pytest.raises(RmsError):
+        api.rmsnorm_train_fwd(x, w, y=x)                     # y over x
+    with pytest.raises(TypeError):
+        api.rmsnorm_train_fwd(x.float(), w)
