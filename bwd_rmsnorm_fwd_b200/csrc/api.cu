@@ -35,6 +35,10 @@ int cuda_fail(cudaError_t e, const char* what) {
 constexpr int kMaxH = 8192;
 constexpr int kFoldSegments = 16;
 constexpr size_t kWsHeader = 256;  // status word, ticket
+// The FP64 accumulator of the non-deterministic combine is kept zero between calls.  It
+// is reserved for the widest row so that the deterministic chunk partials, which follow
+// it, never land on it whatever the H of the call that wrote them.
+constexpr size_t kAccBytes = (size_t)kMaxH * 8;
 
 int64_t g_small_rows_override = -1;
 
@@ -148,7 +152,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t ws_bytes(const rms_shape& s, int det) {
     const int64_t R = s.T * s.heads;
-    size_t b = kWsHeader + align256((size_t)s.H * 8);
+    size_t b = kWsHeader + kAccBytes;
     if (det && !use_small(R, s.H)) b += (size_t)det_plan(R, s.H).n_chunks * s.H * 8;
     return b;
 }
@@ -218,7 +222,7 @@ int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const fl
     p.status = reinterpret_cast<unsigned*>(base);
     p.ticket = reinterpret_cast<unsigned*>(base + 4);
     p.acc = reinterpret_cast<double*>(base + kWsHeader);
-    p.part = reinterpret_cast<double*>(base + kWsHeader + align256((size_t)H * 8));
+    p.part = reinterpret_cast<double*>(base + kWsHeader + kAccBytes);
     const Plan plan = det_plan(R, H);
     p.block_rows = plan.B;
     p.blocks_per_chunk = plan.L;
@@ -241,6 +245,11 @@ int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const fl
 }  // namespace
 
 namespace rmsk {
+
+int set_error(int code, const char* msg) {
+    g_err = msg;
+    return code;
+}
 
 int device_sm_count() {
     static int cached[64];

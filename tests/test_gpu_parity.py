@@ -194,3 +194,23 @@ def test_alias_and_dtype_errors_with_device_tensors():
         api.rmsnorm_train_fwd(x, w, y=x)                     # y over x
     with pytest.raises(TypeError):
         api.rmsnorm_train_fwd(x.float(), w)
+
+
+def test_workspace_shared_by_modes_and_widths():
+    """One workspace serves deterministic calls (chunk partials) and non-deterministic calls
+    (a zero-between-calls FP64 accumulator) of any width, interleaved, without either
+    corrupting the other."""
+    ws = api.Workspace("cuda")
+    cases = []
+    for T, H in [(40000, 256), (9000, 6144), (70000, 512), (5000, 4096)]:
+        x = synth.rows(12, "x", T, H)
+        dy = synth.rows(12, "dy", T, H)
+        w = synth.weight(12, H, "fp32")
+        _, rstd = oracle.train_fwd(x, w)
+        _, ref = oracle.train_bwd(x, w, rstd, dy, want_dx=False)
+        cases.append((dev_rows(x), dev_rows(dy), dev_weight(w), torch.from_numpy(rstd).cuda(), ref))
+    for _ in range(2):
+        for det in (True, False, True):
+            for xd, dyd, wd, rs, ref in cases:
+                _, dw = api.rmsnorm_train_bwd(xd, wd, rs, dyd, deterministic=det, workspace=ws)
+                assert_dw(dw.cpu().numpy(), ref, f"det={det} H={xd.shape[1]}")
