@@ -49,6 +49,8 @@ SIGNATURES = [
     ("rms_residual_train_bwd", _i32,
      [RmsShape, RmsRows, _vp, _i32, _vp, RmsRows, RmsRows, RmsRows, _vp, _i32, _vp, _sz, _i32,
       _vp]),
+    ("rms_train_bwd_noalloc", _i32,
+     [RmsShape, RmsRows, _vp, _i32, _vp, RmsRows, RmsRows, _vp, _vp]),
     ("rms_train_bwd_workspace_bytes", _sz, [RmsShape, _i32, _i32]),
     ("rms_det_plan", _i32, [RmsShape, ctypes.POINTER(ctypes.c_int32),
                             ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),

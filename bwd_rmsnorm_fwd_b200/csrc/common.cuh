@@ -70,6 +70,8 @@ cudaError_t launch_bwd_nondet(const BwdParams& p, bool residual, bool w32, int g
 // (the blocks of one deterministic chunk).  Also the chunk's block count.
 int bwd_slots_for_width(int H);
 int device_sm_count();
+// Records `msg` as this thread's rms_last_error() text and returns `code`.
+int set_error(int code, const char* msg);
 
 }  // namespace rmsk
 

@@ -113,6 +113,23 @@ int rms_residual_train_bwd(rms_shape shape, rms_rows h, const void* w, int w_dty
                            float* dw, int deterministic, void* workspace,
                            size_t workspace_bytes, int grid_ctas, void* stream);
 
+/* Backward without any device allocation: the deterministic == 0 backward of
+ * rms_train_bwd, whose scratch (status word, CTA ticket and FP64 accumulators for up to
+ * 8192 columns: 65,792 bytes) lives in one fixed device array inside this library
+ * instead of a caller-allocated workspace.  The pages have no counterpart; it exists for
+ * callers that cannot allocate device memory at all -- code running inside an
+ * allocator's callbacks, runtimes that hand out only pre-planned buffers, plugins whose
+ * host owns every device buffer -- and so cannot provide a workspace.  The caller still
+ * passes every input and output.  H above 8192 is rejected with RMS_EINVAL.  The first
+ * call on each device looks up the array's device address (cudaGetSymbolAddress with
+ * that device current); make that first call before any stream capture.  Each call
+ * clears the scratch it uses on `stream`, and every GPU that loaded the library keeps
+ * the array until the process exits.  All calls share the one array, so calls whose
+ * work overlaps on the GPU (other streams, unordered threads) race and corrupt dw.
+ * Other arguments, checks and outputs are those of rms_train_bwd. */
+int rms_train_bwd_noalloc(rms_shape shape, rms_rows x, const void* w, int w_dtype,
+                          const float* rstd, rms_rows dy, rms_rows dx, float* dw, void* stream);
+
 /* Workspace bytes the backward needs for this shape, mode and grid (0 on bad input). */
 size_t rms_train_bwd_workspace_bytes(rms_shape shape, int deterministic, int grid_ctas);
 
