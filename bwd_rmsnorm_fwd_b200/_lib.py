@@ -56,6 +56,7 @@ SIGNATURES = [
                             ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),
     ("rms_train_bwd_path", _i32, [RmsShape, _i32]),
     ("rms_set_small_rows_limit", _i64, [_i64]),
+    ("rms_set_wait_limit_cycles", _i64, [_i64]),
     ("rms_status", _i32, [_vp, _vp]),
     ("rms_last_error", ctypes.c_char_p, []),
     ("rms_device_sms", _i32, []),

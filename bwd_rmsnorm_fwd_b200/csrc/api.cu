@@ -41,6 +41,7 @@ constexpr size_t kWsHeader = 256;  // status word, ticket
 constexpr size_t kAccBytes = (size_t)kMaxH * 8;
 
 int64_t g_small_rows_override = -1;
+int64_t g_wait_cycles = rmsk::kDefaultWaitCycles;
 
 struct Span {
     uintptr_t lo, hi;  // [lo, hi)
@@ -228,6 +229,7 @@ int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const fl
     p.blocks_per_chunk = plan.L;
     p.fold_segments = plan.S;
     p.n_chunks = plan.n_chunks;
+    p.wait_cycles = g_wait_cycles;
     const bool res = dh != nullptr;
     const bool w32 = w_dtype == RMS_FP32;
     cudaError_t e;
@@ -378,6 +380,12 @@ int rms_train_bwd_path(rms_shape shape, int deterministic) {
 int64_t rms_set_small_rows_limit(int64_t rows) {
     const int64_t prev = g_small_rows_override;
     g_small_rows_override = rows < 0 ? -1 : rows;
+    return prev;
+}
+
+int64_t rms_set_wait_limit_cycles(int64_t cycles) {
+    const int64_t prev = g_wait_cycles;
+    g_wait_cycles = cycles < 0 ? rmsk::kDefaultWaitCycles : cycles;
     return prev;
 }
 

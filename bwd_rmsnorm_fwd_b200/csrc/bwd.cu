@@ -17,7 +17,7 @@
 //   grid or on the SM count.  Three programs produce exactly these bits:
 //     - bwd_small_kernel: one launch; row tasks compute dx, column tasks walk every
 //       row of a 64-column strip and do the whole fold (used for small row counts);
-//     - bwd_large_kernel<DET> + bwd_fold_kernel: CTAs take whole chunks (each slot of
+//     - bwd_staged_kernel<DET> + bwd_fold_kernel: CTAs take whole chunks (each slot of
 //       the CTA one block), write FP64 chunk partials to the workspace, and the fold
 //       kernel (launched with programmatic dependent launch) finishes the order.
 // * non-deterministic: each CTA takes a contiguous row range; every thread sums eight
@@ -26,12 +26,11 @@
 //   workspace vector with atomics.  The last CTA to finish (atomic ticket) rounds the
 //   vector to FP32 dw and clears it for the next call.
 //
-// The large kernels give each CTA L "slots" of SW warps; a slot owns one row at a time
-// and every thread of the slot owns VPT 16-byte column vectors, so the dw state of a
-// column stays in one thread's registers for the whole block.  The per-row dot
+// The large kernel gives each CTA L "slots" of SW consumer warps; a slot owns one row at
+// a time and every thread of the slot owns VPT 16-byte column vectors, so the dw state of
+// a column stays in one thread's registers for the whole block.  The per-row dot
 // product is a warp-shuffle tree plus, for multi-warp slots, a named barrier over the
-// slot's warps with a double-buffered shared exchange.  P rows are loaded before any
-// is used.
+// slot's warps with a double-buffered shared exchange.
 #include "common.cuh"
 
 namespace rmsk {
@@ -41,154 +40,356 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
 }
 
 // ============================================================================================
-// Large-row kernel: deterministic chunk partials or non-deterministic grid combine.
+// Large-row kernel: a bulk-copy pipeline.  Warp 0 streams the rows of each tile (x, dy
+// and, in the residual form, dh) into a ring of shared-memory stages with cp.async.bulk,
+// one mbarrier per stage counting the bytes; the consumer warps read the stage, compute
+// dx and accumulate dw, and release the stage on a second mbarrier.  The bytes in flight
+// are bounded by shared memory (up to ~200 KB per SM), not by registers.
+//
+// Tiles: a tile holds P consecutive rows of every slot.  Deterministic: CTA c takes chunks
+// c, c + grid, ...; slot s of chunk k owns the block of rows [k*L*B + s*B, +B).
+// Non-deterministic: CTA c takes a contiguous row range, split evenly between slots.
+//
+// Every wait is bounded (BwdParams::wait_cycles).  A wait that gives up sets the status
+// word and a CTA-wide abort flag; from then on consumers stop waiting (control flow stays
+// uniform, so every named barrier is still met) and the producer issues nothing more,
+// then waits for its copies in flight before the CTA exits.
 // ============================================================================================
 
-template <int SW, int VPT, int L, int P, bool DET, bool RES, bool W32>
-__global__ void __launch_bounds__(SW * 32 * L)
-    bwd_large_kernel(const BwdParams p) {
-    constexpr int ST = SW * 32;  // threads per slot
-    constexpr int NT = ST * L;   // threads per CTA
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    double* sm64 = reinterpret_cast<double*>(smem_raw);  // [L][nvec*8]
-    __shared__ float red[L][2][P][SW];
+constexpr int kMaxStages = 16;
+constexpr int kStagedHeader = 1024;  // barriers, flags, slot reduction buffers
 
-    const int tid = threadIdx.x;
-    const int slot = tid / ST;
-    const int ts = tid - slot * ST;
-    const int wis = ts >> 5;
-    const int lane = tid & 31;
+struct StagedCfg {
+    int32_t n_stages;
+    int32_t stage_bytes;   // one stage, all tensors
+    int32_t tensor_bytes;  // one tensor's rows inside a stage
+    int32_t xch_offset;    // FP64 [L][nvec*8] exchange / accumulators
+    int32_t stage_offset;
+};
+
+template <int SW, int VPT, int L, int P, bool DET, bool RES, bool W32>
+__global__ void __launch_bounds__(32 * (1 + SW * L), 1)
+    bwd_staged_kernel(const BwdParams p, const StagedCfg sc) {
+    constexpr int ST = SW * 32;      // threads per slot
+    constexpr int NCW = SW * L;      // consumer warps
+    constexpr int NCT = NCW * 32;    // consumer threads
+    constexpr int RT = L * P;        // rows per stage
+    constexpr int NTEN = RES ? 3 : 2;
+    constexpr int kAllConsumers = 15;  // named barrier over every consumer thread
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);  // full[kMaxStages], empty[kMaxStages]
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 16 * kMaxStages);
+    volatile unsigned* last_flag = reinterpret_cast<volatile unsigned*>(smem + 16 * kMaxStages + 4);
+    float* red = reinterpret_cast<float*>(smem + 16 * kMaxStages + 16);  // [L][2][P][SW]
+    double* xch = reinterpret_cast<double*>(smem + sc.xch_offset);       // [L][nvec*8]
+    unsigned char* stages = smem + sc.stage_offset;
+
+    const int NS = sc.n_stages;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
     const int H = p.H;
     const int nvec = p.nvec;
-    const float Hf = (float)H;
-    double* my64 = sm64 + (size_t)slot * nvec * 8;
+    const uint32_t row_bytes = (uint32_t)H * 2u;
+    const int64_t limit = p.wait_cycles;
+    auto full_bar = [&](int s) { return smem_addr(&bars[s]); };
+    auto empty_bar = [&](int s) { return smem_addr(&bars[kMaxStages + s]); };
 
-    // this thread's weights (FP32)
-    float wv[VPT][8];
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), NCW);
+        }
+        *abort_flag = 0;
+        *last_flag = 0;
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    // ---- the unit sequence (chunks or the CTA's row range), identical for all warps ----
+    const int B = p.block_rows;
+    const int CH = B * L;
+    int64_t lo = 0, hi = 0;
+    if constexpr (!DET) {
+        lo = (int64_t)p.R * blockIdx.x / gridDim.x;
+        hi = (int64_t)p.R * (blockIdx.x + 1) / gridDim.x;
+    }
+    const int n_units = DET ? (p.n_chunks > (int)blockIdx.x
+                                   ? (p.n_chunks - 1 - (int)blockIdx.x) / (int)gridDim.x + 1
+                                   : 0)
+                            : 1;
+    // first row and end row of slot s in unit u
+    auto slot_base = [&](int u, int s) -> int {
+        if constexpr (DET) {
+            const int k = (int)blockIdx.x + u * (int)gridDim.x;
+            return k * CH + s * B;
+        } else {
+            return (int)(lo + (hi - lo) * s / L);
+        }
+    };
+    auto slot_end = [&](int u, int s) -> int {
+        if constexpr (DET) {
+            return min(slot_base(u, s) + B, p.R);
+        } else {
+            return (int)(lo + (hi - lo) * (s + 1) / L);
+        }
+    };
+    auto unit_tiles = [&](int u) -> int {
+        int m = 0;
+#pragma unroll
+        for (int s = 0; s < L; ++s) m = max(m, slot_end(u, s) - slot_base(u, s));
+        return (m + P - 1) / P;
+    };
+
+    if (warp == 0) {
+        // ================= producer =================
+        int j = 0;
+        for (int u = 0; u < n_units; ++u) {
+            int base[L], endr[L];
+#pragma unroll
+            for (int s = 0; s < L; ++s) { base[s] = slot_base(u, s); endr[s] = slot_end(u, s); }
+            const int nt = unit_tiles(u);
+            for (int t = 0; t < nt; ++t, ++j) {
+                const int stage = j % NS;
+                const uint32_t ph = (uint32_t)(j / NS) & 1u;
+                if (j >= NS) {
+                    if (!mbar_wait_bounded(empty_bar(stage), ph ^ 1u, limit)) {
+                        if (lane == 0) { *abort_flag = 1; atomicOr(p.status, kStatusTimeout); }
+                    }
+                }
+                __syncwarp();
+                if (*abort_flag) goto drain;
+                uint32_t bytes = 0;
+#pragma unroll
+                for (int s = 0; s < L; ++s)
+#pragma unroll
+                    for (int q = 0; q < P; ++q)
+                        if (base[s] + t * P + q < endr[s]) bytes += row_bytes * NTEN;
+                if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), bytes);
+                __syncwarp();
+                const uint32_t sbase = smem_addr(stages + (size_t)stage * sc.stage_bytes);
+                for (int c = lane; c < RT * NTEN; c += 32) {
+                    const int ten = c / RT;
+                    const int rr = c - ten * RT;
+                    const int s = rr / P;
+                    const int q = rr - s * P;
+                    const int row = base[s] + t * P + q;
+                    if (row < endr[s]) {
+                        const RowsIn& src = ten == 0 ? p.x : (ten == 1 ? p.dy : p.dh);
+                        bulk_load(sbase + (uint32_t)ten * sc.tensor_bytes + (uint32_t)rr * row_bytes,
+                                  src.ptr + row_offset(row, p.heads, src.st, src.sk), row_bytes,
+                                  full_bar(stage));
+                    }
+                }
+                __syncwarp();
+            }
+        }
+    drain:
+        // every copy issued lands before the CTA may exit (bounded, with the default
+        // limit even when a shorter one was requested)
+        if (lane == 0) {
+            const int last = j;  // tiles issued
+            for (int i = 0; i < NS && i < last; ++i) {
+                const int jj = last - 1 - i;
+                mbar_wait_bounded(full_bar(jj % NS), (uint32_t)(jj / NS) & 1u,
+                                  limit > kDefaultWaitCycles ? limit : kDefaultWaitCycles);
+            }
+        }
+        return;
+    }
+
+    // ================= consumers =================
+    // Packed-pair arithmetic on -xh: every product is formed with nx = x * (-rstd), which
+    // is exactly -xh (round-to-nearest is sign-symmetric), so the deterministic TwoSum
+    // state holds exactly the negation of the documented order's state and is negated
+    // back when a block is converted to FP64.
+    const int ctid = threadIdx.x - 32;
+    const int slot = ctid / ST;
+    const int ts = ctid - slot * ST;
+    const int wis = ts >> 5;
+    const float invH = 1.0f / (float)H;
+    double* my64 = xch + (size_t)slot * nvec * 8;
+    const float2 m1 = make_float2(-1.f, -1.f);
+
+    float2 w2[VPT][4];
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
         const int v = ts + ST * i;
+        float wf[8];
         if (v < nvec) {
-            load_w8<W32>(p.w, 8 * v, wv[i]);
+            load_w8<W32>(p.w, 8 * v, wf);
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) wv[i][e] = 0.f;
+            for (int e = 0; e < 8; ++e) wf[e] = 0.f;
         }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w2[i][k] = make_float2(wf[2 * k], wf[2 * k + 1]);
     }
-
-    float s_[VPT][8], c_[VPT][8];  // DET: TwoSum state; NONDET: s_ = eight-row block sum
-    int buf = 0;
-
-    auto zero_state = [&]() {
+    // DET: (s, c) TwoSum state of -dw.  NONDET: s = eight-row FP32 block of -dw and acc,
+    // the FP64 total of dw.
+    float2 s2[VPT][4], c2[VPT][DET ? 4 : 1];
+    double acc[DET ? 1 : VPT][DET ? 1 : 8];
+    if constexpr (!DET) {
 #pragma unroll
         for (int i = 0; i < VPT; ++i)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) { s_[i][e] = 0.f; c_[i][e] = 0.f; }
-    };
-
-    // Process rows r .. r+P-1 of this slot (rows >= r_end are padding).
-    auto do_rows = [&](int r, int r_end) {
-        uint4 xv[P][VPT], dyv[P][VPT];
-        uint4 dhv[RES ? P : 1][VPT];
-        float rs[P];
-        int64_t odx[P];
+            for (int e = 0; e < 8; ++e) acc[i][e] = 0.0;
+    }
+    int buf = 0;
+    int j = 0;
+    int in_block = 0;
+    // rstd of the next tile, loaded one tile ahead
+    float rs_next[P];
+    {
+        const int b0 = n_units > 0 ? slot_base(0, slot) : 0;
+        const int e0 = n_units > 0 ? slot_end(0, slot) : 0;
 #pragma unroll
-        for (int q = 0; q < P; ++q) {
-            const int rr = r + q;
-            const bool rv = rr < r_end;
-            const int64_t ox = rv ? row_offset(rr, p.heads, p.x.st, p.x.sk) : 0;
-            const int64_t ody = rv ? row_offset(rr, p.heads, p.dy.st, p.dy.sk) : 0;
-            odx[q] = rv ? row_offset(rr, p.heads, p.dx.st, p.dx.sk) : 0;
-            rs[q] = rv ? __ldg(p.rstd + rr) : 0.f;
+        for (int q = 0; q < P; ++q) rs_next[q] = (b0 + q < e0) ? __ldg(p.rstd + b0 + q) : 0.f;
+    }
+    for (int u = 0; u < n_units; ++u) {
+        const int base = slot_base(u, slot);
+        const int endr = slot_end(u, slot);
+        const int nt = unit_tiles(u);
 #pragma unroll
-            for (int i = 0; i < VPT; ++i) {
-                const int v = ts + ST * i;
-                const bool ok = rv && v < nvec;
-                xv[q][i] = ok ? ld_stream16(p.x.ptr + ox + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
-                dyv[q][i] = ok ? ld_stream16(p.dy.ptr + ody + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+        for (int i = 0; i < VPT; ++i)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                s2[i][k] = make_float2(0.f, 0.f);
+                if constexpr (DET) c2[i][k] = make_float2(0.f, 0.f);
             }
-            if constexpr (RES) {
-                const int64_t odh = rv ? row_offset(rr, p.heads, p.dh.st, p.dh.sk) : 0;
+        for (int t = 0; t < nt; ++t, ++j) {
+            const int stage = j % NS;
+            const uint32_t ph = (uint32_t)(j / NS) & 1u;
+            float rs[P];
+#pragma unroll
+            for (int q = 0; q < P; ++q) rs[q] = rs_next[q];
+            {   // prefetch the next tile's rstd (next unit's first tile at the end of a unit)
+                int nb = base + (t + 1) * P, ne = endr;
+                if (t + 1 == nt) {
+                    nb = u + 1 < n_units ? slot_base(u + 1, slot) : 0;
+                    ne = u + 1 < n_units ? slot_end(u + 1, slot) : 0;
+                }
+#pragma unroll
+                for (int q = 0; q < P; ++q) rs_next[q] = (nb + q < ne) ? __ldg(p.rstd + nb + q) : 0.f;
+            }
+            if (!*abort_flag) {
+                if (!mbar_wait_bounded(full_bar(stage), ph, limit)) {
+                    *abort_flag = 1;
+                    if (lane == 0) atomicOr(p.status, kStatusTimeout);
+                }
+            }
+            const unsigned char* sb = stages + (size_t)stage * sc.stage_bytes;
+            const uint4* sx = reinterpret_cast<const uint4*>(sb + (size_t)(slot * P) * row_bytes);
+            const uint4* sdy = reinterpret_cast<const uint4*>(sb + sc.tensor_bytes +
+                                                              (size_t)(slot * P) * row_bytes);
+            const uint4* sdh = reinterpret_cast<const uint4*>(sb + 2 * sc.tensor_bytes +
+                                                              (size_t)(slot * P) * row_bytes);
+            // pass 1: per-thread partial sums of g * (-xh)
+            float dot[P];
+#pragma unroll
+            for (int q = 0; q < P; ++q) {
+                const float2 nrs = make_float2(-rs[q], -rs[q]);
+                float2 d2 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int i = 0; i < VPT; ++i) {
                     const int v = ts + ST * i;
-                    const bool ok = rv && v < nvec;
-                    dhv[q][i] = ok ? ld_stream16(p.dh.ptr + odh + 8 * v)
-                                   : make_uint4(0u, 0u, 0u, 0u);
-                }
-            }
-        }
-        // per-thread partial dot products sum_j g_j xh_j
-        float dot[P];
+                    if (v < nvec) {
+                        const uint4 xr = sx[q * nvec + v];
+                        const uint4 dr = sdy[q * nvec + v];
+                        const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+                        const uint32_t dw4[4] = {dr.x, dr.y, dr.z, dr.w};
 #pragma unroll
-        for (int q = 0; q < P; ++q) {
-            float d = 0.f;
-#pragma unroll
-            for (int i = 0; i < VPT; ++i) {
-                float xf[8], gf[8];
-                unpack8(xv[q][i], xf);
-                unpack8(dyv[q][i], gf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    d = __fmaf_rn(__fmul_rn(gf[e], wv[i][e]), __fmul_rn(xf[e], rs[q]), d);
-            }
-            dot[q] = warp_sum(d);
-        }
-        if constexpr (SW > 1) {
-            if (lane == 0) {
-#pragma unroll
-                for (int q = 0; q < P; ++q) red[slot][buf][q][wis] = dot[q];
-            }
-            named_bar(1 + slot, ST);
-#pragma unroll
-            for (int q = 0; q < P; ++q) {
-                float d = 0.f;
-#pragma unroll
-                for (int w2 = 0; w2 < SW; ++w2) d = __fadd_rn(d, red[slot][buf][q][w2]);
-                dot[q] = d;
-            }
-            buf ^= 1;
-        }
-        // dx and the dw accumulation, rows in increasing order
-#pragma unroll
-        for (int q = 0; q < P; ++q) {
-            if (r + q >= r_end) continue;
-            const float cr = __fdiv_rn(dot[q], Hf);
-#pragma unroll
-            for (int i = 0; i < VPT; ++i) {
-                const int v = ts + ST * i;
-                if (v >= nvec) continue;
-                float xf[8], df[8], out[8];
-                unpack8(xv[q][i], xf);
-                unpack8(dyv[q][i], df);
-                float hf[8];
-                if constexpr (RES) unpack8(dhv[q][i], hf);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float xh = __fmul_rn(xf[e], rs[q]);
-                    const float g = __fmul_rn(df[e], wv[i][e]);
-                    float o = __fmul_rn(rs[q], __fmaf_rn(-xh, cr, g));
-                    if constexpr (RES) o = __fadd_rn(o, hf[e]);
-                    out[e] = o;
-                    if constexpr (DET) {
-                        twosum_product(df[e], xh, s_[i][e], c_[i][e]);
-                    } else {
-                        s_[i][e] = __fmaf_rn(df[e], xh, s_[i][e]);
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 nx = mul2(bf16x2_to_f2(xw[k]), nrs);
+                            const float2 g = mul2(bf16x2_to_f2(dw4[k]), w2[i][k]);
+                            d2 = fma2(g, nx, d2);
+                        }
                     }
                 }
-                st16(p.dx.ptr + odx[q] + 8 * v, pack8(out));
+                dot[q] = warp_sum(d2.x + d2.y);
+            }
+            if constexpr (SW > 1) {
+                if (lane == 0) {
+#pragma unroll
+                    for (int q = 0; q < P; ++q) red[((slot * 2 + buf) * P + q) * SW + wis] = dot[q];
+                }
+                named_bar(1 + slot, ST);
+#pragma unroll
+                for (int q = 0; q < P; ++q) {
+                    float d = 0.f;
+#pragma unroll
+                    for (int w2i = 0; w2i < SW; ++w2i) d += red[((slot * 2 + buf) * P + q) * SW + w2i];
+                    dot[q] = d;
+                }
+                buf ^= 1;
+            }
+            // pass 2: dx = rstd (g - xh c) = rstd (g + nx c), c = -dot / H; dw, rows in order
+#pragma unroll
+            for (int q = 0; q < P; ++q) {
+                if (base + t * P + q >= endr) continue;
+                const float cr = -dot[q] * invH;
+                const float2 c2v = make_float2(cr, cr);
+                const float2 rs2 = make_float2(rs[q], rs[q]);
+                const float2 nrs = make_float2(-rs[q], -rs[q]);
+                const int row = base + t * P + q;
+                uint16_t* dxrow = p.dx.ptr + row_offset(row, p.heads, p.dx.st, p.dx.sk);
+#pragma unroll
+                for (int i = 0; i < VPT; ++i) {
+                    const int v = ts + ST * i;
+                    if (v >= nvec) continue;
+                    const uint4 xr = sx[q * nvec + v];
+                    const uint4 dr = sdy[q * nvec + v];
+                    const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+                    const uint32_t dw4[4] = {dr.x, dr.y, dr.z, dr.w};
+                    uint32_t hw[4] = {0u, 0u, 0u, 0u};
+                    if constexpr (RES) {
+                        const uint4 hr = sdh[q * nvec + v];
+                        hw[0] = hr.x; hw[1] = hr.y; hw[2] = hr.z; hw[3] = hr.w;
+                    }
+                    uint32_t out[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 d = bf16x2_to_f2(dw4[k]);
+                        const float2 nx = mul2(bf16x2_to_f2(xw[k]), nrs);
+                        const float2 g = mul2(d, w2[i][k]);
+                        float2 o = mul2(fma2(nx, c2v, g), rs2);
+                        if constexpr (RES) o = add2(o, bf16x2_to_f2(hw[k]));
+                        out[k] = pack2(o);
+                        if constexpr (DET) {
+                            // -p, its exact error e (fma(-d, -xh, -p) = d xh - p), TwoSum
+                            const float2 np = mul2(d, nx);
+                            const float2 e = fma2(mul2(d, m1), nx, np);
+                            const float2 tt = add2(s2[i][k], np);
+                            const float2 z = sub2(tt, s2[i][k]);
+                            const float2 err = add2(sub2(s2[i][k], sub2(tt, z)), sub2(np, z));
+                            c2[i][k] = add2(c2[i][k], sub2(err, e));
+                            s2[i][k] = tt;
+                        } else {
+                            s2[i][k] = fma2(d, nx, s2[i][k]);
+                        }
+                    }
+                    st16(dxrow + 8 * v, make_uint4(out[0], out[1], out[2], out[3]));
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty_bar(stage));
+            if constexpr (!DET) {
+                // eight-row FP32 blocks go into the FP64 total
+                in_block += P;
+                if (in_block >= 8 || t + 1 == nt) {
+#pragma unroll
+                    for (int i = 0; i < VPT; ++i)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            acc[i][2 * k] -= (double)s2[i][k].x;
+                            acc[i][2 * k + 1] -= (double)s2[i][k].y;
+                            s2[i][k] = make_float2(0.f, 0.f);
+                        }
+                    in_block = 0;
+                }
             }
         }
-    };
-
-    if constexpr (DET) {
-        const int B = p.block_rows;
-        const int CH = B * L;
-        for (int k = blockIdx.x; k < p.n_chunks; k += gridDim.x) {
-            const int row0 = k * CH + slot * B;
-            const int row_end = min(row0 + B, p.R);
-            zero_state();
-            for (int r = row0; r < row_end; r += P) do_rows(r, row_end);
+        if constexpr (DET) {
+            const int k = (int)blockIdx.x + u * (int)gridDim.x;
             const int nb = min(L, (p.R - k * CH + B - 1) / B);  // non-empty blocks of chunk k
             if constexpr (L == 1) {
 #pragma unroll
@@ -197,11 +398,11 @@ __global__ void __launch_bounds__(SW * 32 * L)
                     if (v >= nvec) continue;
                     double* dst = p.part + (size_t)k * H + 8 * v;
 #pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        double2 t;
-                        t.x = (double)s_[i][e] + (double)c_[i][e];
-                        t.y = (double)s_[i][e + 1] + (double)c_[i][e + 1];
-                        *reinterpret_cast<double2*>(dst + e) = t;
+                    for (int kk = 0; kk < 4; ++kk) {
+                        double2 t2;
+                        t2.x = -((double)s2[i][kk].x + (double)c2[i][kk].x);
+                        t2.y = -((double)s2[i][kk].y + (double)c2[i][kk].y);
+                        *reinterpret_cast<double2*>(dst + 2 * kk) = t2;
                     }
                 }
             } else {
@@ -211,75 +412,56 @@ __global__ void __launch_bounds__(SW * 32 * L)
                         const int v = ts + ST * i;
                         if (v >= nvec) continue;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            my64[8 * v + e] = (double)s_[i][e] + (double)c_[i][e];
+                        for (int kk = 0; kk < 4; ++kk) {
+                            my64[8 * v + 2 * kk] = -((double)s2[i][kk].x + (double)c2[i][kk].x);
+                            my64[8 * v + 2 * kk + 1] = -((double)s2[i][kk].y + (double)c2[i][kk].y);
+                        }
                     }
                 }
-                __syncthreads();
-                for (int col = tid; col < H; col += NT) {
-                    double a = sm64[col];
-                    for (int b = 1; b < nb; ++b) a += sm64[(size_t)b * nvec * 8 + col];
+                named_bar(kAllConsumers, NCT);
+                for (int col = ctid; col < H; col += NCT) {
+                    double a = xch[col];
+                    for (int b = 1; b < nb; ++b) a += xch[(size_t)b * nvec * 8 + col];
                     p.part[(size_t)k * H + col] = a;
                 }
-                __syncthreads();
+                named_bar(kAllConsumers, NCT);
             }
         }
-        // let the fold kernel start its launch; it waits for this grid to finish
+    }
+    if constexpr (DET) {
+        // let the fold kernel begin launching; it waits for this grid to complete
         asm volatile("griddepcontrol.launch_dependents;");
     } else {
-        // contiguous row range of this CTA, split evenly between its slots
-        const int64_t lo = (int64_t)p.R * blockIdx.x / gridDim.x;
-        const int64_t hi = (int64_t)p.R * (blockIdx.x + 1) / gridDim.x;
-        const int slo = (int)(lo + (hi - lo) * slot / L);
-        const int shi = (int)(lo + (hi - lo) * (slot + 1) / L);
+        // slot totals meet in shared memory (the stage ring, free once every tile is
+        // consumed), then one FP64 atomic per column per CTA
+        double* tot = reinterpret_cast<double*>(stages);
+        named_bar(kAllConsumers, NCT);
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int v = ts + ST * i;
-            if (v < nvec)
+            if (v >= nvec) continue;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) my64[8 * v + e] = 0.0;
+            for (int e = 0; e < 8; ++e) tot[(size_t)slot * nvec * 8 + 8 * v + e] = acc[i][e];
         }
-        zero_state();
-        constexpr int kBlock = 8;  // rows per FP32 block
-        static_assert(kBlock % P == 0, "P must divide the block");
-        int in_block = 0;
-        for (int r = slo; r < shi; r += P) {
-            do_rows(r, shi);
-            in_block += P;
-            if (in_block == kBlock || r + P >= shi) {
+        named_bar(kAllConsumers, NCT);
+        for (int col = ctid; col < H; col += NCT) {
+            double a = tot[col];
 #pragma unroll
-                for (int i = 0; i < VPT; ++i) {
-                    const int v = ts + ST * i;
-                    if (v >= nvec) continue;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        my64[8 * v + e] += (double)s_[i][e];
-                        s_[i][e] = 0.f;
-                    }
-                }
-                in_block = 0;
-            }
-        }
-        __syncthreads();
-        for (int col = tid; col < H; col += NT) {
-            double a = sm64[col];
-#pragma unroll
-            for (int b = 1; b < L; ++b) a += sm64[(size_t)b * nvec * 8 + col];
+            for (int b = 1; b < L; ++b) a += tot[(size_t)b * nvec * 8 + col];
             atomicAdd(p.acc + col, a);
         }
         __threadfence();
-        __syncthreads();
-        __shared__ unsigned last;
-        if (tid == 0) last = (atomicAdd(p.ticket, 1u) == gridDim.x - 1) ? 1u : 0u;
-        __syncthreads();
-        if (last) {
+        named_bar(kAllConsumers, NCT);
+        if (ctid == 0) *last_flag = (atomicAdd(p.ticket, 1u) == gridDim.x - 1) ? 1u : 0u;
+        named_bar(kAllConsumers, NCT);
+        if (*last_flag) {
             __threadfence();
-            for (int col = tid; col < H; col += NT) {
+            for (int col = ctid; col < H; col += NCT) {
                 const double a = __ldcg(p.acc + col);
                 p.dw[col] = __double2float_rn(a);
                 p.acc[col] = 0.0;
             }
-            if (tid == 0) *p.ticket = 0u;
+            if (ctid == 0) *p.ticket = 0u;
         }
     }
 }
@@ -466,37 +648,41 @@ __global__ void __launch_bounds__(kSmallThreads) bwd_small_kernel(const BwdParam
 
 namespace {
 
-template <typename K>
-int occupancy(K kern, int threads, size_t smem) {
-    int o = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, threads, smem) != cudaSuccess)
-        return 1;
-    return o > 0 ? o : 1;
-}
 
 template <int SW, int VPT, int L, int P, bool DET, bool RES, bool W32>
 cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
-    auto kern = bwd_large_kernel<SW, VPT, L, P, DET, RES, W32>;
-    constexpr int NT = SW * 32 * L;
-    const size_t smem = (DET && L == 1) ? 0 : (size_t)L * p.nvec * 8 * sizeof(double);
-    static int occ_cached = -1;
+    auto kern = bwd_staged_kernel<SW, VPT, L, P, DET, RES, W32>;
+    constexpr int NT = 32 * (1 + SW * L);
+    constexpr int NTEN = RES ? 3 : 2;
+    constexpr size_t kBudget = 220 * 1024;
+    StagedCfg sc;
+    const size_t xch = (DET && L > 1) ? (size_t)L * p.nvec * 8 * sizeof(double) : 0;
+    sc.xch_offset = kStagedHeader;
+    sc.stage_offset = (int32_t)(kStagedHeader + ((xch + 127) & ~size_t(127)));
+    sc.tensor_bytes = L * P * p.H * 2;
+    sc.stage_bytes = NTEN * sc.tensor_bytes;
+    int ns = (int)((kBudget - sc.stage_offset) / sc.stage_bytes);
+    if (ns > kMaxStages) ns = kMaxStages;
+    if (ns < 2) return cudaErrorInvalidConfiguration;
+    if (!DET && (size_t)ns * sc.stage_bytes < (size_t)L * p.nvec * 8 * sizeof(double))
+        return cudaErrorInvalidConfiguration;  // the slot totals must fit in the ring
+    sc.n_stages = ns;
+    const size_t smem = (size_t)sc.stage_offset + (size_t)ns * sc.stage_bytes;
     static size_t smem_set = 0;
-    if (smem != 0 && smem > smem_set) {
+    if (smem > smem_set) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
         smem_set = smem;
-        occ_cached = -1;
     }
-    if (occ_cached < 0) occ_cached = occupancy(kern, NT, smem);
     int grid = grid_ctas;
     if (grid <= 0) {
-        const int64_t cap = (int64_t)device_sm_count() * occ_cached;
+        const int64_t cap = device_sm_count();
         int64_t need = DET ? p.n_chunks : ((int64_t)p.R + L * 8 - 1) / (L * 8);
         if (need < 1) need = 1;
         grid = (int)(need < cap ? need : cap);
     }
-    kern<<<grid, NT, smem, s>>>(p);
+    kern<<<grid, NT, smem, s>>>(p, sc);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || !DET) return e;
     // fold kernel, programmatic dependent launch
@@ -513,7 +699,8 @@ cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, bwd_fold_kernel, p);
 }
 
-// Slot layout per width: SW warps per slot, VPT vectors per thread, L slots per CTA.
+// Slot layout per width: SW warps per slot, VPT vectors per thread, L slots per CTA, P rows
+// of a slot per stage.  L is also the block count of a deterministic chunk.
 template <bool DET, bool RES, bool W32>
 cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     const int nv = p.nvec;

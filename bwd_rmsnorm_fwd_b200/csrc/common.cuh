@@ -52,10 +52,14 @@ struct BwdParams {
     int32_t blocks_per_chunk;
     int32_t fold_segments;
     int32_t n_chunks;
+    // limit of every device-side wait, in SM clock cycles
+    int64_t wait_cycles;
 };
 
 // device status bits
 constexpr unsigned kStatusTimeout = 1u;
+// default limit of a device-side wait (about two seconds at 2 GHz)
+constexpr int64_t kDefaultWaitCycles = 4000000000LL;
 
 // ---- host-side launchers (defined in fwd.cu / bwd.cu) -------------------------------------
 
@@ -139,6 +143,20 @@ __device__ __forceinline__ void load_w8(const void* w, int e, float (&f)[8]) {
     }
 }
 
+// ---- packed FP32 pairs (sm_100 f32x2 instructions; each lane rounds like the scalar op) ----
+
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+// a - b, exactly one rounding (fma with -1 is exact before the rounding)
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    return __ffma2_rn(b, make_float2(-1.f, -1.f), a);
+}
+__device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16x2(v.x, v.y); }
+
 __device__ __forceinline__ int64_t row_offset(int32_t r, int32_t heads, int64_t st,
                                               int64_t sk) {
     if (heads == 1) return (int64_t)r * st;
@@ -165,6 +183,78 @@ __device__ __forceinline__ void twosum_product(float a, float b, float& s, float
     const float err = __fadd_rn(__fsub_rn(s, __fsub_rn(t, z)), __fsub_rn(p, z));
     c = __fadd_rn(c, __fadd_rn(err, e));
     s = t;
+}
+
+// ---- shared-memory barriers and bulk copies (sm_90+ PTX) -----------------------------------
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// make barrier initialisation visible to the bulk-copy (async) proxy
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Non-blocking probe of the phase of `parity`.
+__device__ __forceinline__ bool mbar_probe(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Waits for the phase of `parity` to complete; gives up after `limit` SM cycles and
+// returns false.  Never waits forever.  A limit of 0 is a single non-blocking probe
+// (try_wait itself may suspend the thread for a while before returning).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int64_t limit) {
+    if (limit <= 0) return mbar_probe(bar, parity);
+    if (mbar_test(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_test(bar, parity)) return true;
+        if (clock64() - t0 > limit) return false;
+    }
+}
+
+// Bulk copy global -> shared (this CTA), completion counted in bytes on `bar`.
+// dst, src and bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
 }
 
 }  // namespace rmsk
