@@ -15,7 +15,7 @@ from . import _lib
 
 __all__ = [
     "rmsnorm_train_fwd", "rmsnorm_train_bwd", "Workspace", "det_plan", "bwd_path",
-    "set_small_rows_limit", "status",
+    "set_small_rows_limit", "status", "forward_status",
 ]
 
 
@@ -149,7 +149,15 @@ def set_small_rows_limit(rows: int) -> int:
 
 
 def status(workspace: Workspace | None = None, device=None) -> None:
+    """Raises RmsError if a backward on this workspace (the default one if None) recorded
+    a device-side error; clears the word."""
     ws = workspace or _workspace_for(device if device is not None else "cuda")
     if ws.buf.numel() == 0:
         return
     _lib.check(_lib.lib().rms_status(ws.buf.data_ptr(), _stream()))
+
+
+def forward_status() -> None:
+    """Raises RmsError if a forward on the current device recorded a device-side error;
+    clears the word."""
+    _lib.check(_lib.lib().rms_status(None, _stream()))

@@ -297,6 +297,7 @@ int rms_train_fwd(rms_shape shape, rms_rows x, const void* w, int w_dtype, rms_r
     p.w = w;
     p.rstd = rstd;
     p.eps = eps;
+    p.wait_cycles = g_wait_cycles;
     cudaError_t e = rmsk::launch_fwd(p, false, w_dtype == RMS_FP32, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "forward launch");
 }
@@ -333,6 +334,7 @@ int rms_residual_train_fwd(rms_shape shape, rms_rows x, rms_rows residual, const
     p.w = w;
     p.rstd = rstd;
     p.eps = eps;
+    p.wait_cycles = g_wait_cycles;
     cudaError_t e = rmsk::launch_fwd(p, true, w_dtype == RMS_FP32, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "residual forward launch");
 }
@@ -390,16 +392,23 @@ int64_t rms_set_wait_limit_cycles(int64_t cycles) {
 }
 
 int rms_status(void* workspace, void* stream) {
-    if (!workspace) return fail(RMS_EINVAL, "workspace is null");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaStreamSynchronize(st);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
     unsigned word = 0;
-    e = cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+    cudaError_t e;
+    if (!workspace) {
+        e = rmsk::fwd_status_take(st, &word);
+        if (e != cudaSuccess) return cuda_fail(e, "reading the forward status word");
+    } else {
+        e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+        e = cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+        if (word) {
+            e = cudaMemset(workspace, 0, sizeof word);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status)");
+        }
+    }
     if (word) {
-        e = cudaMemset(workspace, 0, sizeof word);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status)");
         if (word & rmsk::kStatusTimeout)
             return fail(RMS_ETIMEOUT, "a device-side bounded wait gave up (status 0x%x)", word);
         return fail(RMS_ECUDA, "device status 0x%x", word);

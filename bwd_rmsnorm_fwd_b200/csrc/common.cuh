@@ -28,6 +28,7 @@ struct FwdParams {
     const void* w;
     float* rstd;
     float eps;
+    int64_t wait_cycles;  // limit of every device-side wait, in SM clock cycles
 };
 
 struct BwdParams {
@@ -74,6 +75,9 @@ cudaError_t launch_bwd_nondet(const BwdParams& p, bool residual, bool w32, int g
 // (the blocks of one deterministic chunk).  Also the chunk's block count.
 int bwd_slots_for_width(int H);
 int device_sm_count();
+// Reads and clears the forward's device status word (a library global on the current
+// device); synchronises `s` first.
+cudaError_t fwd_status_take(cudaStream_t s, unsigned* word);
 // Records `msg` as this thread's rms_last_error() text and returns `code`.
 int set_error(int code, const char* msg);
 

@@ -12,11 +12,17 @@
 // loads of a group are issued before any use, which keeps VPT*ROWS*16 bytes per lane
 // in flight.  Squares of BF16 values are exact in FP32; each 16-byte vector is summed
 // as a small tree, lanes sequentially over their vectors, then a 5-level shuffle tree.
+// rstd = rsqrtf(sum * (1/H) + eps) in FP32: CUDA documents rsqrtf to within 2 ulp, and
+// the FMA rounds the mean once, so rstd is within a few FP32 ulps of the exact value.
 #include "common.cuh"
 
 namespace rmsk {
 
 constexpr int kFwdThreads = 256;
+
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 template <int VPT, int ROWS, bool RES, bool W32>
 __global__ void __launch_bounds__(kFwdThreads) fwd_kernel(const FwdParams p) {
@@ -24,7 +30,7 @@ __global__ void __launch_bounds__(kFwdThreads) fwd_kernel(const FwdParams p) {
     const int gwarp = (int)((blockIdx.x * kFwdThreads + threadIdx.x) >> 5);
     const int nwarps = (int)((gridDim.x * kFwdThreads) >> 5);
     const int ngroups = (p.R + ROWS - 1) / ROWS;
-    const float Hf = (float)p.H;
+    const float invH = 1.0f / (float)p.H;
 
     for (int g = gwarp; g < ngroups; g += nwarps) {
         const int r0 = g * ROWS;
@@ -90,8 +96,7 @@ __global__ void __launch_bounds__(kFwdThreads) fwd_kernel(const FwdParams p) {
                 acc = __fadd_rn(acc, __fadd_rn(__fadd_rn(s01, s23), __fadd_rn(s45, s67)));
             }
             const float ss = warp_sum(acc);
-            const float ms = __fdiv_rn(ss, Hf);
-            rs[q] = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, p.eps)));
+            rs[q] = rsqrtf(__fmaf_rn(ss, invH, p.eps));
         }
 #pragma unroll
         for (int q = 0; q < ROWS; ++q) {
@@ -115,6 +120,218 @@ __global__ void __launch_bounds__(kFwdThreads) fwd_kernel(const FwdParams p) {
         for (int q = 1; q < ROWS; ++q)
             if (lane == q) mine = rs[q];
         if (lane < ROWS && r0 + lane < p.R) p.rstd[r0 + lane] = mine;
+    }
+}
+
+// ---- wide rows: bulk-copy pipeline ------------------------------------------------------------
+// Warp 0 streams P rows per slot (x, and the residual in the residual form) into a ring of
+// shared-memory stages with cp.async.bulk; L slots of SW consumer warps each own one row
+// at a time: sum of squares (packed FP32 pairs), a shuffle tree plus a named barrier over
+// the slot's warps, then y = (x * rstd) * w stored straight to global memory.  The CTA
+// takes a contiguous row range split evenly between its slots.  Waits are bounded; a wait
+// that gives up sets the status word and the pipeline stops waiting (see the backward).
+
+// status word of the forward kernels (they take no workspace); read by rms_status(NULL, .)
+__device__ unsigned g_fwd_status;
+
+constexpr int kFwdMaxStages = 16;
+constexpr int kFwdHeader = 512;
+
+struct FwdStaged {
+    int32_t n_stages;
+    int32_t stage_bytes;
+    int32_t tensor_bytes;
+};
+
+template <int SW, int VPT, int L, int P, bool RES, bool W32>
+__global__ void __launch_bounds__(32 * (1 + SW * L), 1)
+    fwd_staged_kernel(const FwdParams p, const FwdStaged sc) {
+    constexpr int ST = SW * 32;
+    constexpr int NCW = SW * L;
+    constexpr int RT = L * P;
+    constexpr int NTEN = RES ? 2 : 1;
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 16 * kFwdMaxStages);
+    float* red = reinterpret_cast<float*>(smem + 16 * kFwdMaxStages + 16);  // [L][2][P][SW]
+    unsigned char* stages = smem + kFwdHeader;
+    const int NS = sc.n_stages;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int H = p.H;
+    const int nvec = p.nvec;
+    const uint32_t row_bytes = (uint32_t)H * 2u;
+    const int64_t limit = p.wait_cycles;
+    auto full_bar = [&](int s) { return smem_addr(&bars[s]); };
+    auto empty_bar = [&](int s) { return smem_addr(&bars[kFwdMaxStages + s]); };
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), NCW);
+        }
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    __syncthreads();
+    const int64_t lo = (int64_t)p.R * blockIdx.x / gridDim.x;
+    const int64_t hi = (int64_t)p.R * (blockIdx.x + 1) / gridDim.x;
+    auto sbase = [&](int s) { return (int)(lo + (hi - lo) * s / L); };
+    int maxlen = 0;
+#pragma unroll
+    for (int s = 0; s < L; ++s) maxlen = max(maxlen, sbase(s + 1) - sbase(s));
+    const int nt = (maxlen + P - 1) / P;
+
+    if (warp == 0) {
+        int base[L], endr[L];
+#pragma unroll
+        for (int s = 0; s < L; ++s) { base[s] = sbase(s); endr[s] = sbase(s + 1); }
+        int j = 0;
+        for (; j < nt; ++j) {
+            const int stage = j % NS;
+            const uint32_t ph = (uint32_t)(j / NS) & 1u;
+            if (j >= NS && !mbar_wait_bounded(empty_bar(stage), ph ^ 1u, limit)) {
+                if (lane == 0) { *abort_flag = 1; atomicOr(&g_fwd_status, kStatusTimeout); }
+            }
+            __syncwarp();
+            if (*abort_flag) break;
+            uint32_t bytes = 0;
+#pragma unroll
+            for (int s = 0; s < L; ++s)
+#pragma unroll
+                for (int q = 0; q < P; ++q)
+                    if (base[s] + j * P + q < endr[s]) bytes += row_bytes * NTEN;
+            if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), bytes);
+            __syncwarp();
+            const uint32_t sb = smem_addr(stages + (size_t)stage * sc.stage_bytes);
+            for (int c = lane; c < RT * NTEN; c += 32) {
+                const int ten = c / RT;
+                const int rr = c - ten * RT;
+                const int s = rr / P;
+                const int q = rr - s * P;
+                const int row = base[s] + j * P + q;
+                if (row < endr[s]) {
+                    const RowsIn& src = ten == 0 ? p.x : p.res;
+                    bulk_load(sb + (uint32_t)ten * sc.tensor_bytes + (uint32_t)rr * row_bytes,
+                              src.ptr + row_offset(row, p.heads, src.st, src.sk), row_bytes,
+                              full_bar(stage));
+                }
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            for (int i = 0; i < NS && i < j; ++i) {
+                const int jj = j - 1 - i;
+                mbar_wait_bounded(full_bar(jj % NS), (uint32_t)(jj / NS) & 1u,
+                                  limit > kDefaultWaitCycles ? limit : kDefaultWaitCycles);
+            }
+        }
+        return;
+    }
+
+    const int ctid = threadIdx.x - 32;
+    const int slot = ctid / ST;
+    const int ts = ctid - slot * ST;
+    const int wis = ts >> 5;
+    const int base = sbase(slot);
+    const int endr = sbase(slot + 1);
+    const float invH = 1.0f / (float)H;
+    float2 w2[VPT][4];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int v = ts + ST * i;
+        float wf[8];
+        if (v < nvec) {
+            load_w8<W32>(p.w, 8 * v, wf);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) wf[e] = 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w2[i][k] = make_float2(wf[2 * k], wf[2 * k + 1]);
+    }
+    int buf = 0;
+    for (int t = 0; t < nt; ++t) {
+        const int stage = t % NS;
+        const uint32_t ph = (uint32_t)(t / NS) & 1u;
+        if (!*abort_flag && !mbar_wait_bounded(full_bar(stage), ph, limit)) {
+            *abort_flag = 1;
+            if (lane == 0) atomicOr(&g_fwd_status, kStatusTimeout);
+        }
+        const unsigned char* sbp = stages + (size_t)stage * sc.stage_bytes;
+        const uint4* sx = reinterpret_cast<const uint4*>(sbp + (size_t)(slot * P) * row_bytes);
+        const uint4* sr = reinterpret_cast<const uint4*>(sbp + sc.tensor_bytes +
+                                                         (size_t)(slot * P) * row_bytes);
+        uint4 hv[RES ? P : 1][RES ? VPT : 1];
+        float ss[P];
+#pragma unroll
+        for (int q = 0; q < P; ++q) {
+            const int row = base + t * P + q;
+            const bool ok = row < endr;
+            float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int v = ts + ST * i;
+                if (v < nvec) {
+                    uint4 xr = sx[q * nvec + v];
+                    if constexpr (RES) {
+                        // h = BF16(x + residual); the norm runs on the rounded h
+                        const uint4 rr = sr[q * nvec + v];
+                        xr.x = pack2(add2(bf16x2_to_f2(xr.x), bf16x2_to_f2(rr.x)));
+                        xr.y = pack2(add2(bf16x2_to_f2(xr.y), bf16x2_to_f2(rr.y)));
+                        xr.z = pack2(add2(bf16x2_to_f2(xr.z), bf16x2_to_f2(rr.z)));
+                        xr.w = pack2(add2(bf16x2_to_f2(xr.w), bf16x2_to_f2(rr.w)));
+                        hv[q][i] = xr;
+                        if (ok) st16(p.h.ptr + row_offset(row, p.heads, p.h.st, p.h.sk) + 8 * v, xr);
+                    }
+                    const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 x2 = bf16x2_to_f2(xw[k]);
+                        a2 = fma2(x2, x2, a2);  // squares of BF16 values are exact
+                    }
+                }
+            }
+            ss[q] = warp_sum(a2.x + a2.y);
+        }
+        if constexpr (SW > 1) {
+            if (lane == 0) {
+#pragma unroll
+                for (int q = 0; q < P; ++q) red[((slot * 2 + buf) * P + q) * SW + wis] = ss[q];
+            }
+            named_bar(1 + slot, ST);
+#pragma unroll
+            for (int q = 0; q < P; ++q) {
+                float a = 0.f;
+#pragma unroll
+                for (int w = 0; w < SW; ++w) a += red[((slot * 2 + buf) * P + q) * SW + w];
+                ss[q] = a;
+            }
+            buf ^= 1;
+        }
+#pragma unroll
+        for (int q = 0; q < P; ++q) {
+            const int row = base + t * P + q;
+            if (row >= endr) continue;
+            const float rstd = rsqrtf(__fmaf_rn(ss[q], invH, p.eps));
+            const float2 rs2 = make_float2(rstd, rstd);
+            uint16_t* yrow = p.y.ptr + row_offset(row, p.heads, p.y.st, p.y.sk);
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int v = ts + ST * i;
+                if (v >= nvec) continue;
+                uint4 xr;
+                if constexpr (RES) xr = hv[q][i]; else xr = sx[q * nvec + v];
+                const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+                uint32_t out[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    out[k] = pack2(mul2(mul2(bf16x2_to_f2(xw[k]), rs2), w2[i][k]));
+                st16(yrow + 8 * v, make_uint4(out[0], out[1], out[2], out[3]));
+            }
+            if (ts == 0) p.rstd[row] = rstd;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(stage));
     }
 }
 
@@ -156,10 +373,67 @@ cudaError_t launch_vpt(const FwdParams& p, bool res, bool w32, cudaStream_t s) {
     return w32 ? launch_one<VPT, 1, false, true>(p, s) : launch_one<VPT, 1, false, false>(p, s);
 }
 
+template <int SW, int VPT, int L, int P, bool RES, bool W32>
+cudaError_t launch_staged(const FwdParams& p, cudaStream_t s) {
+    auto kern = fwd_staged_kernel<SW, VPT, L, P, RES, W32>;
+    constexpr int NT = 32 * (1 + SW * L);
+    constexpr size_t kBudget = 220 * 1024;
+    FwdStaged sc;
+    sc.tensor_bytes = L * P * p.H * 2;
+    sc.stage_bytes = (RES ? 2 : 1) * sc.tensor_bytes;
+    int ns = (int)((kBudget - kFwdHeader) / sc.stage_bytes);
+    if (ns > kFwdMaxStages) ns = kFwdMaxStages;
+    if (ns < 2) return cudaErrorInvalidConfiguration;
+    sc.n_stages = ns;
+    const size_t smem = kFwdHeader + (size_t)ns * sc.stage_bytes;
+    static size_t smem_set = 0;
+    if (smem > smem_set) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        smem_set = smem;
+    }
+    int64_t need = ((int64_t)p.R + L * 4 - 1) / (L * 4);
+    const int64_t cap = device_sm_count();
+    const int grid = (int)(need < cap ? need : cap);
+    kern<<<grid, NT, smem, s>>>(p, sc);
+    return cudaGetLastError();
+}
+
+template <bool RES, bool W32>
+cudaError_t dispatch_staged(const FwdParams& p, cudaStream_t s) {
+    const int nv = p.nvec;
+    if (nv <= 32) return launch_staged<1, 1, 8, 4, RES, W32>(p, s);
+    if (nv <= 64) return launch_staged<1, 2, 8, 2, RES, W32>(p, s);
+    if (nv <= 128) return launch_staged<2, 2, 4, 2, RES, W32>(p, s);
+    if (nv <= 192) return launch_staged<2, 3, 4, 2, RES, W32>(p, s);
+    if (nv <= 256) return launch_staged<4, 2, 2, 2, RES, W32>(p, s);
+    if (nv <= 384) return launch_staged<4, 3, 2, 2, RES, W32>(p, s);
+    if (nv <= 512) return launch_staged<8, 2, 1, 2, RES, W32>(p, s);
+    if (nv <= 768) return launch_staged<8, 3, 1, 2, RES, W32>(p, s);
+    return launch_staged<8, 4, 1, 2, RES, W32>(p, s);
+}
+
 }  // namespace
+
+// Rows below this count take the register kernel: too few rows per SM to fill a pipeline.
+constexpr int kFwdStagedMinRowsPerSm = 16;
+
+cudaError_t fwd_status_take(cudaStream_t s, unsigned* word) {
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(word, g_fwd_status, sizeof(unsigned));
+    if (e != cudaSuccess || !*word) return e;
+    const unsigned zero = 0;
+    return cudaMemcpyToSymbol(g_fwd_status, &zero, sizeof zero);
+}
 
 cudaError_t launch_fwd(const FwdParams& p, bool res, bool w32, cudaStream_t s) {
     if (p.R <= 0) return cudaSuccess;
+    if ((int64_t)p.R >= (int64_t)kFwdStagedMinRowsPerSm * device_sm_count()) {
+        if (res) return w32 ? dispatch_staged<true, true>(p, s) : dispatch_staged<true, false>(p, s);
+        return w32 ? dispatch_staged<false, true>(p, s) : dispatch_staged<false, false>(p, s);
+    }
     const int need = (p.nvec + 31) / 32;  // vectors per lane
     if (need <= 1) return launch_vpt<1, 4>(p, res, w32, s);
     if (need <= 2) return launch_vpt<2, 2>(p, res, w32, s);

@@ -155,17 +155,18 @@ int rms_train_bwd_path(rms_shape shape, int deterministic);
  * the default.  Returns the previous override (-1 if none). */
 int64_t rms_set_small_rows_limit(int64_t rows);
 
-/* Limit, in SM clock cycles, of every device-side wait of later backward launches in
- * this process (the bulk-copy pipeline's barrier waits); the default is about two
- * seconds.  A wait that reaches it makes the kernel record RMS_ETIMEOUT in the workspace
- * status word (see rms_status) and finish without waiting further; its dx/dw are then
- * invalid.  Shorter limits exist to test that path (0 makes every wait a single
+/* Limit, in SM clock cycles, of every device-side wait of later launches in this
+ * process (the bulk-copy pipelines' barrier waits); the default is about two seconds.  A
+ * wait that reaches it makes the kernel record RMS_ETIMEOUT in its status word (see
+ * rms_status) and finish without waiting further; its outputs are then invalid.  Shorter limits exist to test that path (0 makes every wait a single
  * non-blocking probe); a negative value restores the default.  Returns the previous
  * limit.  Not thread-safe against concurrent launches. */
 int64_t rms_set_wait_limit_cycles(int64_t cycles);
 
-/* Synchronises `stream`, reads and clears the device status word of `workspace`.
- * Returns RMS_OK, RMS_ETIMEOUT or RMS_ECUDA. */
+/* Synchronises `stream`, reads and clears the device status word of `workspace` (the
+ * backward's), or, with workspace == NULL, the forward's status word (one per device,
+ * inside the library: the forward takes no workspace).  Returns RMS_OK, RMS_ETIMEOUT or
+ * RMS_ECUDA. */
 int rms_status(void* workspace, void* stream);
 
 /* Message for the last non-zero return on this thread ("" if none). */

@@ -6,9 +6,9 @@ atol 1e-4 + rtol 1e-4 against FP64), plus, for outputs the pages fix only by dty
 y within one BF16 ulp of the oracle's correctly rounded value (the GPU rounds an FP32
 product whose error is ~3e-7 relative, so it can land on the other side of a rounding
 boundary but never further), rstd within 2e-6 relative (FP32 sum of exact squares: a
-tree of depth <= 40 gives <= 40 * 2^-24 relative on the mean, half of that on rstd,
-plus two correctly rounded operations), h bit-exact (the sum of two BF16 values is
-exact in FP32 whenever it can matter, so one rounding gives the oracle's bits).
+summation depth <= 40 gives <= 40 * 2^-24 relative on the mean, half of that on rstd,
+plus one rounding of the scaled mean and rsqrtf's documented 2 ulp), h bit-exact (the
+sum of two BF16 values is exact in FP32 whenever it can matter, so one rounding gives the oracle's bits).
 """
 
 from __future__ import annotations
