@@ -76,6 +76,8 @@ __global__ void __launch_bounds__(32 * (1 + SW * L), 1)
     constexpr int RT = L * P;        // rows per stage
     constexpr int NTEN = RES ? 3 : 2;
     constexpr int kAllConsumers = 15;  // named barrier over every consumer thread
+    static_assert(16 * kMaxStages + 16 + L * 2 * P * SW * 4 <= kStagedHeader,
+                  "slot reduction buffers must fit in the header");
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);  // full[kMaxStages], empty[kMaxStages]
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 16 * kMaxStages);
@@ -167,14 +169,28 @@ __global__ void __launch_bounds__(32 * (1 + SW * L), 1)
                 if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), bytes);
                 __syncwarp();
                 const uint32_t sbase = smem_addr(stages + (size_t)stage * sc.stage_bytes);
+                // one copy per (tensor, slot) when rows are contiguous, else one per row
+                for (int c = lane; c < L * NTEN; c += 32) {
+                    const int ten = c / L;
+                    const int s = c - ten * L;
+                    const RowsIn& src = ten == 0 ? p.x : (ten == 1 ? p.dy : p.dh);
+                    if (!rows_contiguous(src, p.heads, H)) continue;
+                    const int row0 = base[s] + t * P;
+                    const int n = min(P, endr[s] - row0);
+                    if (n > 0)
+                        bulk_load(sbase + (uint32_t)ten * sc.tensor_bytes +
+                                      (uint32_t)(s * P) * row_bytes,
+                                  src.ptr + row_offset(row0, p.heads, src.st, src.sk),
+                                  (uint32_t)n * row_bytes, full_bar(stage));
+                }
                 for (int c = lane; c < RT * NTEN; c += 32) {
                     const int ten = c / RT;
                     const int rr = c - ten * RT;
                     const int s = rr / P;
                     const int q = rr - s * P;
                     const int row = base[s] + t * P + q;
-                    if (row < endr[s]) {
-                        const RowsIn& src = ten == 0 ? p.x : (ten == 1 ? p.dy : p.dh);
+                    const RowsIn& src = ten == 0 ? p.x : (ten == 1 ? p.dy : p.dh);
+                    if (row < endr[s] && !rows_contiguous(src, p.heads, H)) {
                         bulk_load(sbase + (uint32_t)ten * sc.tensor_bytes + (uint32_t)rr * row_bytes,
                                   src.ptr + row_offset(row, p.heads, src.st, src.sk), row_bytes,
                                   full_bar(stage));
@@ -699,20 +715,31 @@ cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, bwd_fold_kernel, p);
 }
 
-// Slot layout per width: SW warps per slot, VPT vectors per thread, L slots per CTA, P rows
-// of a slot per stage.  L is also the block count of a deterministic chunk.
+// Rows of a slot per stage: 4 when two such stages fit beside the exchange area, else 2.
+template <int SW, int VPT, int L, bool DET, bool RES, bool W32>
+cudaError_t launch_large_p(const BwdParams& p, int grid_ctas, cudaStream_t s) {
+    constexpr size_t kRoom = 220 * 1024 - kStagedHeader;
+    const size_t xch = (DET && L > 1) ? (size_t)L * p.nvec * 8 * sizeof(double) : 0;
+    const size_t row = (size_t)(RES ? 3 : 2) * L * p.H * 2;
+    if (2 * 4 * row + xch + 128 <= kRoom)
+        return launch_large<SW, VPT, L, 4, DET, RES, W32>(p, grid_ctas, s);
+    return launch_large<SW, VPT, L, 2, DET, RES, W32>(p, grid_ctas, s);
+}
+
+// Slot layout per width: SW warps per slot, VPT vectors per thread, L slots per CTA.  L is
+// also the block count of a deterministic chunk.
 template <bool DET, bool RES, bool W32>
 cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     const int nv = p.nvec;
-    if (nv <= 32) return launch_large<1, 1, 8, 2, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 64) return launch_large<1, 2, 8, 2, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 128) return launch_large<2, 2, 4, 2, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 192) return launch_large<2, 3, 4, 2, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 256) return launch_large<4, 2, 2, 2, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 384) return launch_large<4, 3, 2, 2, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 512) return launch_large<8, 2, 1, 2, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 768) return launch_large<8, 3, 1, 2, DET, RES, W32>(p, grid_ctas, s);
-    return launch_large<8, 4, 1, 2, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 32) return launch_large_p<1, 1, 8, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 64) return launch_large_p<1, 2, 8, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 128) return launch_large_p<2, 2, 4, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 192) return launch_large_p<2, 3, 4, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 256) return launch_large_p<4, 2, 2, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 384) return launch_large_p<4, 3, 2, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 512) return launch_large_p<8, 2, 1, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 768) return launch_large_p<8, 3, 1, DET, RES, W32>(p, grid_ctas, s);
+    return launch_large_p<8, 4, 1, DET, RES, W32>(p, grid_ctas, s);
 }
 
 template <int VPT, bool RES, bool W32>

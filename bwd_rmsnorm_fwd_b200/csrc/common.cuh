@@ -169,6 +169,12 @@ __device__ __forceinline__ int64_t row_offset(int32_t r, int32_t heads, int64_t 
     return (int64_t)t * st + (int64_t)k * sk;
 }
 
+// True when consecutive rows of the view follow each other in memory (row r + 1 starts
+// where row r ends), so a run of rows is one contiguous byte range.
+__device__ __forceinline__ bool rows_contiguous(const RowsIn& v, int32_t heads, int32_t H) {
+    return heads == 1 ? v.st == H : (v.sk == H && v.st == (int64_t)heads * H);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);

@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kFwdThreads) fwd_kernel(const FwdParams p) {
 __device__ unsigned g_fwd_status;
 
 constexpr int kFwdMaxStages = 16;
-constexpr int kFwdHeader = 512;
+constexpr int kFwdHeader = 2048;  // barriers (256 B), flags (16 B), slot reduction buffers
 
 struct FwdStaged {
     int32_t n_stages;
@@ -150,6 +150,8 @@ __global__ void __launch_bounds__(32 * (1 + SW * L), 1)
     constexpr int NCW = SW * L;
     constexpr int RT = L * P;
     constexpr int NTEN = RES ? 2 : 1;
+    static_assert(16 * kFwdMaxStages + 16 + L * 2 * P * SW * 4 <= kFwdHeader,
+                  "slot reduction buffers must fit in the header");
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 16 * kFwdMaxStages);
@@ -203,14 +205,27 @@ __global__ void __launch_bounds__(32 * (1 + SW * L), 1)
             if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), bytes);
             __syncwarp();
             const uint32_t sb = smem_addr(stages + (size_t)stage * sc.stage_bytes);
+            // one copy per (tensor, slot) when rows are contiguous, else one per row
+            for (int c = lane; c < L * NTEN; c += 32) {
+                const int ten = c / L;
+                const int s = c - ten * L;
+                const RowsIn& src = ten == 0 ? p.x : p.res;
+                if (!rows_contiguous(src, p.heads, H)) continue;
+                const int row0 = base[s] + j * P;
+                const int n = min(P, endr[s] - row0);
+                if (n > 0)
+                    bulk_load(sb + (uint32_t)ten * sc.tensor_bytes + (uint32_t)(s * P) * row_bytes,
+                              src.ptr + row_offset(row0, p.heads, src.st, src.sk),
+                              (uint32_t)n * row_bytes, full_bar(stage));
+            }
             for (int c = lane; c < RT * NTEN; c += 32) {
                 const int ten = c / RT;
                 const int rr = c - ten * RT;
                 const int s = rr / P;
                 const int q = rr - s * P;
                 const int row = base[s] + j * P + q;
-                if (row < endr[s]) {
-                    const RowsIn& src = ten == 0 ? p.x : p.res;
+                const RowsIn& src = ten == 0 ? p.x : p.res;
+                if (row < endr[s] && !rows_contiguous(src, p.heads, H)) {
                     bulk_load(sb + (uint32_t)ten * sc.tensor_bytes + (uint32_t)rr * row_bytes,
                               src.ptr + row_offset(row, p.heads, src.st, src.sk), row_bytes,
                               full_bar(stage));
@@ -400,18 +415,29 @@ cudaError_t launch_staged(const FwdParams& p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Rows of a slot per stage: the largest of 8, 4, 2 that leaves room for two stages (the
+// larger the tile, the more rows each barrier, reduction and wait is spread over).
+template <int SW, int VPT, int L, bool RES, bool W32>
+cudaError_t launch_staged_p(const FwdParams& p, cudaStream_t s) {
+    constexpr size_t kRoom = 220 * 1024 - kFwdHeader;
+    const size_t row = (size_t)(RES ? 2 : 1) * L * p.H * 2;
+    if (2 * 8 * row <= kRoom) return launch_staged<SW, VPT, L, 8, RES, W32>(p, s);
+    if (2 * 4 * row <= kRoom) return launch_staged<SW, VPT, L, 4, RES, W32>(p, s);
+    return launch_staged<SW, VPT, L, 2, RES, W32>(p, s);
+}
+
 template <bool RES, bool W32>
 cudaError_t dispatch_staged(const FwdParams& p, cudaStream_t s) {
     const int nv = p.nvec;
-    if (nv <= 32) return launch_staged<1, 1, 8, 4, RES, W32>(p, s);
-    if (nv <= 64) return launch_staged<1, 2, 8, 2, RES, W32>(p, s);
-    if (nv <= 128) return launch_staged<2, 2, 4, 2, RES, W32>(p, s);
-    if (nv <= 192) return launch_staged<2, 3, 4, 2, RES, W32>(p, s);
-    if (nv <= 256) return launch_staged<4, 2, 2, 2, RES, W32>(p, s);
-    if (nv <= 384) return launch_staged<4, 3, 2, 2, RES, W32>(p, s);
-    if (nv <= 512) return launch_staged<8, 2, 1, 2, RES, W32>(p, s);
-    if (nv <= 768) return launch_staged<8, 3, 1, 2, RES, W32>(p, s);
-    return launch_staged<8, 4, 1, 2, RES, W32>(p, s);
+    if (nv <= 32) return launch_staged_p<1, 1, 8, RES, W32>(p, s);
+    if (nv <= 64) return launch_staged_p<1, 2, 8, RES, W32>(p, s);
+    if (nv <= 128) return launch_staged_p<2, 2, 4, RES, W32>(p, s);
+    if (nv <= 192) return launch_staged_p<2, 3, 4, RES, W32>(p, s);
+    if (nv <= 256) return launch_staged_p<4, 2, 2, RES, W32>(p, s);
+    if (nv <= 384) return launch_staged_p<4, 3, 2, RES, W32>(p, s);
+    if (nv <= 512) return launch_staged_p<8, 2, 1, RES, W32>(p, s);
+    if (nv <= 768) return launch_staged_p<8, 3, 1, RES, W32>(p, s);
+    return launch_staged_p<8, 4, 1, RES, W32>(p, s);
 }
 
 }  // namespace
