@@ -251,35 +251,64 @@ def graph_time_us(fn, flush, torch, reps=20):
     return statistics.median(ts)
 
 
+def kernel_time_us(fn, flush, torch, reps=30):
+    """Kernel-active time per call: the summed device durations of this library's kernels
+    (CUPTI records through torch.profiler), L2 flushed before every call, divided by the
+    number of calls.  Used where a call lasts a few microseconds, below what CUDA events
+    around a graph replay resolve."""
+    from torch.profiler import ProfilerActivity, profile
+    fn()
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        for _ in range(reps):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+    total = 0.0
+    for e in prof.key_averages():
+        if "rmsk::" in e.key:
+            t = getattr(e, "device_time_total", None)
+            if t is None:
+                t = getattr(e, "cuda_time_total", 0.0)
+            total += t
+    return total / reps
+
+
 def sweep(torch, api, flush, peak, dev):
     """Per-configuration table: us per call (graph replay, cold L2) and fraction of the
     measured HBM bandwidth, for every BASELINE configuration."""
     out = []
     ws = api.Workspace(dev)
 
-    def rec(cfg, form, H, T, wdt, op, us, nbytes):
+    def rec(cfg, form, H, T, wdt, op, us, nbytes, timer_name):
         gbs = nbytes / (us * 1e-6) / 1e9
         out.append({"cfg": cfg, "form": form, "H": H, "T": T, "w": wdt, "op": op,
-                    "us": round(us, 2), "gbs": round(gbs, 1), "frac": round(gbs / peak, 3)})
+                    "us": round(us, 2), "gbs": round(gbs, 1), "frac": round(gbs / peak, 3),
+                    "timer": timer_name})
 
     def ops(cfg, form, x, dy, w, H, T, R, wdt, heads=1, res=None, dh=None, do=("fwd", "det", "nondet")):
         wb = 2 if wdt == "bf16" else 4
         isres = res is not None
+        # a few microseconds per call: CUPTI kernel time; otherwise graph replay
+        small = R * H <= (1 << 22)
+        tname = "cupti_kernel" if small else "graph_replay"
+        timer = ((lambda fn: kernel_time_us(fn, flush, torch)) if small else
+                 (lambda fn: graph_time_us(fn, flush, torch)))
         if isres:
             h, _, rstd = api.rmsnorm_train_fwd(x, w, residual=res)
         else:
             _, rstd = api.rmsnorm_train_fwd(x, w)
             h = x
         if "fwd" in do:
-            us = graph_time_us(lambda: api.rmsnorm_train_fwd(x, w, residual=res), flush, torch)
-            rec(cfg, form, H, T, wdt, "fwd", us, bytes_fwd(R, H, wb, isres))
+            us = timer(lambda: api.rmsnorm_train_fwd(x, w, residual=res))
+            rec(cfg, form, H, T, wdt, "fwd", us, bytes_fwd(R, H, wb, isres), tname)
         for det in (True, False):
             if ("det" if det else "nondet") not in do:
                 continue
-            us = graph_time_us(lambda: api.rmsnorm_train_bwd(h, w, rstd, dy, deterministic=det,
-                                                             dh=dh, workspace=ws), flush, torch)
+            us = timer(lambda: api.rmsnorm_train_bwd(h, w, rstd, dy, deterministic=det, dh=dh,
+                                                     workspace=ws))
             rec(cfg, form, H, T, wdt, "bwd_det" if det else "bwd_nondet", us,
-                bytes_bwd(R, H, wb, isres))
+                bytes_bwd(R, H, wb, isres), tname)
 
     # Tiny and small-T sweep (deterministic backward, single launch)
     x, dy, w = make_inputs(64, 512, "fp32", 1, dev, torch)
