@@ -37,9 +37,10 @@ if ROOT not in sys.path:
 
 METRIC = "RMSNorm train bwd/fwd us per call and achieved HBM GB/s (% of B200 peak)"
 PAGES_STEP_US = 1640.48  # B200, H6144 T131072 BF16 weight, non-det 2xfwd+bwd (PR #8848 table)
+PAGES_STEP_DET_US = 1637.76  # the same row, deterministic
 FALLBACK_HBM_GBS = 6650.0
 HEAD_T, HEAD_H = 131072, 6144
-WORKLOAD = ("large-T checkpointed step (fwd, fwd recompute, bwd deterministic=False), "
+WORKLOAD = ("large-T checkpointed step (fwd, fwd recompute, bwd), "
             "x/dy BF16 [131072, 6144] N(0,1), BF16 w 1+0.1N(0,1), eps 1e-6")
 
 
@@ -274,7 +275,10 @@ def kernel_time_us(fn, flush, torch, reps=30):
     return total / reps
 
 
-def sweep(torch, api, flush, peak, dev):
+SWEEP_GROUPS = ("tiny", "small-T", "residual", "per-head", "large-T")
+
+
+def sweep(torch, api, flush, peak, dev, groups=SWEEP_GROUPS):
     """Per-configuration table: us per call (graph replay, cold L2) and fraction of the
     measured HBM bandwidth, for every BASELINE configuration."""
     out = []
@@ -311,21 +315,22 @@ def sweep(torch, api, flush, peak, dev):
                 bytes_bwd(R, H, wb, isres), tname)
 
     # Tiny and small-T sweep (deterministic backward, single launch)
-    x, dy, w = make_inputs(64, 512, "fp32", 1, dev, torch)
-    ops("tiny", "plain", x, dy, w, 512, 64, 64, "fp32", do=("fwd", "det"))
-    for H in (256, 512, 2048, 4096):
+    if "tiny" in groups:
+        x, dy, w = make_inputs(64, 512, "fp32", 1, dev, torch)
+        ops("tiny", "plain", x, dy, w, 512, 64, 64, "fp32", do=("fwd", "det"))
+    for H in (256, 512, 2048, 4096) if "small-T" in groups else ():
         for wdt in ("bf16", "fp32"):
             xa, dya, w = make_inputs(227, H, wdt, 2, dev, torch)
             for T in (1, 2, 8, 32, 87, 227):
                 ops("small-T", "plain", xa[:T], dya[:T], w, H, T, T, wdt, do=("det",))
     # residual H 6144
-    for T in (32, 4096, 65537):
+    for T in (32, 4096, 65537) if "residual" in groups else ():
         x, dy, w = make_inputs(T, 6144, "bf16", 3, dev, torch)
         res, dh, _ = make_inputs(T, 6144, "bf16", 4, dev, torch)
         ops("residual", "res", x, dy, w, 6144, T, T, "bf16", res=res, dh=dh)
         del x, dy, res, dh
     # per-head views, FP32 weight
-    for T in (1024, 16384):
+    for T in (1024, 16384) if "per-head" in groups else ():
         for name, heads, st, sk in (("24x256_pages", 24, 12288, 512),
                                     ("24x256_dense", 24, 6144, 256), ("4x256", 4, 1024, 256)):
             n = (T - 1) * st + (heads - 1) * sk + 256
@@ -339,7 +344,7 @@ def sweep(torch, api, flush, peak, dev):
             ops("per-head", name, x, dy, w, 256, T, T * heads, "fp32", heads=heads)
             del bx, bd
     # large T
-    for H in (1536, 2048, 4096, 5120, 6144):
+    for H in (1536, 2048, 4096, 5120, 6144) if "large-T" in groups else ():
         for wdt in ("bf16", "fp32"):
             xa, dya, w = make_inputs(131072, H, wdt, 6, dev, torch)
             for T in (65537, 98304, 131072):
@@ -354,7 +359,10 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--sweep", default="all", choices=["all", "none"])
+    ap.add_argument("--sweep", default="all", choices=["all", "none", *SWEEP_GROUPS],
+                    help="per-configuration table: every group, none, or one group")
+    ap.add_argument("--det", action="store_true",
+                    help="the step's backward uses deterministic=True")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows", type=int, default=HEAD_T, help="T of the headline step")
@@ -394,7 +402,7 @@ def main():
 
     for _ in range(args.warmup):
         rstd = step()
-        api.rmsnorm_train_bwd(x, w, rstd, dy, deterministic=False, workspace=ws)
+        api.rmsnorm_train_bwd(x, w, rstd, dy, deterministic=args.det, workspace=ws)
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
@@ -409,7 +417,7 @@ def main():
         e0.record()
         rstd = step()
         e1.record()
-        api.rmsnorm_train_bwd(x, w, rstd, dy, deterministic=False, workspace=ws)
+        api.rmsnorm_train_bwd(x, w, rstd, dy, deterministic=args.det, workspace=ws)
         e2.record()
         evs.append((e0, e1, e2))
     torch.cuda.synchronize()
@@ -446,7 +454,7 @@ def main():
         dyd.copy_(dyh, non_blocking=True)
         api.rmsnorm_train_fwd(xd, w)
         _, r2 = api.rmsnorm_train_fwd(xd, w)
-        dxd, dwd = api.rmsnorm_train_bwd(xd, w, r2, dyd, deterministic=False, workspace=ws)
+        dxd, dwd = api.rmsnorm_train_bwd(xd, w, r2, dyd, deterministic=args.det, workspace=ws)
         dxh.copy_(dxd, non_blocking=True)
         dwh.copy_(dwd, non_blocking=True)
         b.record()
@@ -457,10 +465,11 @@ def main():
     e2e_us = statistics.median(e2e) if e2e else None
 
     per_cfg = None
-    if args.sweep == "all" and rank == 0:
+    if args.sweep != "none" and rank == 0:
         del x, dy
         torch.cuda.empty_cache()
-        per_cfg = sweep(torch, api, flush, peak, dev)
+        per_cfg = sweep(torch, api, flush, peak, dev,
+                        SWEEP_GROUPS if args.sweep == "all" else (args.sweep,))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -471,11 +480,12 @@ def main():
             "metric": METRIC, "value": round(us_step, 2), "unit": "us", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": False, "scaling": "weak",
-            "vs_baseline": (round(us_step / PAGES_STEP_US, 4)
+            "vs_baseline": (round(us_step / (PAGES_STEP_DET_US if args.det else PAGES_STEP_US), 4)
                             if (R, H) == (HEAD_T, HEAD_H) else None),
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD if (R, H) == (HEAD_T, HEAD_H) else
-                       f"checkpointed step at T={R}, H={H} (reduced case)", "T": R, "H": H,
+            "config": {"workload": (WORKLOAD if (R, H) == (HEAD_T, HEAD_H) else
+                                    f"checkpointed step at T={R}, H={H} (reduced case)")
+                       + f", backward deterministic={args.det}", "T": R, "H": H,
                        "w": "bf16",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2, and L2 flushed before every step"},
@@ -484,13 +494,14 @@ def main():
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": peak_kind,
-                         "kernel": f"bwd_large_kernel (deterministic=False), H{H} T{R}",
+                         "kernel": f"bwd_staged_kernel (deterministic={args.det}), H{H} T{R}",
                          "bytes_per_launch": bwd_bytes, "launch_us": round(bwd_avg_us, 2),
-                         "traffic": recorded_traffic(f"bwd_nondet_h{H}_t{R}_bf16")},
+                         "traffic": recorded_traffic(
+                             f"bwd_{'det' if args.det else 'nondet'}_h{H}_t{R}_bf16")},
             "e2e": {"value": round(e2e_us, 1) if e2e_us else None, "unit": "us",
                     "h2d_bytes_per_step": 2 * R * H * 2,
                     "d2h_bytes_per_step": R * H * 2 + H * 4},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": (4 if args.det else 3) * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }

@@ -57,7 +57,7 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
 // ============================================================================================
 
 constexpr int kMaxStages = 16;
-constexpr int kStagedHeader = 1024;  // barriers, flags, slot reduction buffers
+constexpr int kStagedHeader = 2048;  // barriers, flags, slot reduction buffers
 
 struct StagedCfg {
     int32_t n_stages;
@@ -329,13 +329,10 @@ __global__ void __launch_bounds__(32 * (1 + SW * L), 1)
                     for (int q = 0; q < P; ++q) red[((slot * 2 + buf) * P + q) * SW + wis] = dot[q];
                 }
                 named_bar(1 + slot, ST);
+                // every warp re-reduces the SW partials: one shared load and a shuffle tree
 #pragma unroll
-                for (int q = 0; q < P; ++q) {
-                    float d = 0.f;
-#pragma unroll
-                    for (int w2i = 0; w2i < SW; ++w2i) d += red[((slot * 2 + buf) * P + q) * SW + w2i];
-                    dot[q] = d;
-                }
+                for (int q = 0; q < P; ++q)
+                    dot[q] = warp_sum(lane < SW ? red[((slot * 2 + buf) * P + q) * SW + lane] : 0.f);
                 buf ^= 1;
             }
             // pass 2: dx = rstd (g - xh c) = rstd (g + nx c), c = -dot / H; dw, rows in order
@@ -530,62 +527,87 @@ __global__ void __launch_bounds__(32 * kFoldSegMax) bwd_fold_kernel(const BwdPar
 // Small-row single kernel: row tasks (dx) and column tasks (dw, the full fixed order).
 // ============================================================================================
 
-constexpr int kSmallThreads = 256;
+constexpr int kSmallThreads = 512;
 constexpr int kColStrip = 64;   // columns per column task
 constexpr int kRowBatch = 16;   // rows loaded together by a column-task lane
 
-template <int VPT, bool RES, bool W32>
-__global__ void __launch_bounds__(kSmallThreads) bwd_small_kernel(const BwdParams p,
-                                                                  int n_row_ctas) {
+template <int TPR, int VPT, bool RES, bool W32>
+__global__ void __launch_bounds__(kSmallThreads) bwd_small_kernel(const BwdParams p) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int H = p.H;
-    if ((int)blockIdx.x < n_row_ctas) {
-        // ---- row task: one warp per row ----
-        const int r = blockIdx.x * (kSmallThreads / 32) + warp;
-        if (r >= p.R) return;
-        const int64_t ox = row_offset(r, p.heads, p.x.st, p.x.sk);
-        const int64_t ody = row_offset(r, p.heads, p.dy.st, p.dy.sk);
-        const int64_t odx = row_offset(r, p.heads, p.dx.st, p.dx.sk);
-        const float rs = __ldg(p.rstd + r);
+    // column tasks take the first block indices (they are the longer tasks, so they start
+    // first); row tasks follow
+    const int n_col_ctas = (H + kColStrip - 1) / kColStrip;
+    if ((int)blockIdx.x >= n_col_ctas) {
+        // ---- row task: TPR threads per row (TPR * VPT * 8 >= H), 256 / TPR rows per CTA.
+        // The code stays short (VPT <= 4): when the L2 is cold the kernel's own instructions
+        // come from DRAM, so its size is part of the latency.
+        constexpr int RPC = kSmallThreads / TPR;
+        constexpr int WPR = TPR / 32;
+        __shared__ float red[RPC][WPR > 1 ? WPR : 1];
+        const int rl = threadIdx.x / TPR;
+        const int tr = threadIdx.x - rl * TPR;
+        const int r = ((int)blockIdx.x - n_col_ctas) * RPC + rl;
+        const bool rv = r < p.R;
+        const int64_t ox = rv ? row_offset(r, p.heads, p.x.st, p.x.sk) : 0;
+        const int64_t ody = rv ? row_offset(r, p.heads, p.dy.st, p.dy.sk) : 0;
+        const float rs = rv ? __ldg(p.rstd + r) : 0.f;
         uint4 xv[VPT], dyv[VPT];
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-            const int v = lane + 32 * i;
-            const bool ok = v < p.nvec;
+            const int v = tr + TPR * i;
+            const bool ok = rv && v < p.nvec;
             xv[i] = ok ? ld_stream16(p.x.ptr + ox + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
             dyv[i] = ok ? ld_stream16(p.dy.ptr + ody + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float wf[VPT][8];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int v = tr + TPR * i;
+            if (v < p.nvec) {
+                load_w8<W32>(p.w, 8 * v, wf[i]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) wf[i][e] = 0.f;
+            }
         }
         float d = 0.f;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-            const int v = lane + 32 * i;
-            if (v >= p.nvec) continue;
-            float xf[8], df[8], wf[8];
+            float xf[8], df[8];
             unpack8(xv[i], xf);
             unpack8(dyv[i], df);
-            load_w8<W32>(p.w, 8 * v, wf);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                d = __fmaf_rn(__fmul_rn(df[e], wf[e]), __fmul_rn(xf[e], rs), d);
+                d = __fmaf_rn(__fmul_rn(df[e], wf[i][e]), __fmul_rn(xf[e], rs), d);
         }
-        const float cr = __fdiv_rn(warp_sum(d), (float)H);
+        d = warp_sum(d);
+        if constexpr (WPR > 1) {
+            if (lane == 0) red[rl][warp - rl * WPR] = d;
+            __syncthreads();
+            d = 0.f;
+#pragma unroll
+            for (int w2 = 0; w2 < WPR; ++w2) d += red[rl][w2];
+        }
+        if (!rv) return;
+        const float cr = __fdiv_rn(d, (float)H);
+        const int64_t odx = row_offset(r, p.heads, p.dx.st, p.dx.sk);
         int64_t odh = 0;
         if constexpr (RES) odh = row_offset(r, p.heads, p.dh.st, p.dh.sk);
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-            const int v = lane + 32 * i;
+            const int v = tr + TPR * i;
             if (v >= p.nvec) continue;
-            float xf[8], df[8], wf[8], out[8];
+            float xf[8], df[8], out[8];
             unpack8(xv[i], xf);
             unpack8(dyv[i], df);
-            load_w8<W32>(p.w, 8 * v, wf);
             float hf[8];
             if constexpr (RES) unpack8(ld_stream16(p.dh.ptr + odh + 8 * v), hf);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const float xh = __fmul_rn(xf[e], rs);
-                const float g = __fmul_rn(df[e], wf[e]);
+                const float g = __fmul_rn(df[e], wf[i][e]);
                 float o = __fmul_rn(rs, __fmaf_rn(-xh, cr, g));
                 if constexpr (RES) o = __fadd_rn(o, hf[e]);
                 out[e] = o;
@@ -597,7 +619,7 @@ __global__ void __launch_bounds__(kSmallThreads) bwd_small_kernel(const BwdParam
     // ---- column task: columns [c0, c0 + 64), every row, the whole fixed order ----
     extern __shared__ __align__(16) unsigned char smem_raw[];
     double* bp = reinterpret_cast<double*>(smem_raw);  // [n_blocks][64] block partials
-    const int c0 = ((int)blockIdx.x - n_row_ctas) * kColStrip;
+    const int c0 = (int)blockIdx.x * kColStrip;
     const int j = c0 + 2 * lane;  // this lane's column pair
     const bool jok = j < H;
     const int B = p.block_rows;
@@ -727,7 +749,9 @@ cudaError_t launch_large_p(const BwdParams& p, int grid_ctas, cudaStream_t s) {
 }
 
 // Slot layout per width: SW warps per slot, VPT vectors per thread, L slots per CTA.  L is
-// also the block count of a deterministic chunk.
+// also the block count of a deterministic chunk and depends on the width only; SW and VPT
+// are free (measured per width and mode): the deterministic mode, which carries a TwoSum
+// state per column, runs best with more warps and fewer columns per thread.
 template <bool DET, bool RES, bool W32>
 cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     const int nv = p.nvec;
@@ -735,17 +759,23 @@ cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     if (nv <= 64) return launch_large_p<1, 2, 8, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 128) return launch_large_p<2, 2, 4, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 192) return launch_large_p<2, 3, 4, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 256) return launch_large_p<4, 2, 2, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 256) return launch_large_p<8, 1, 2, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 384) return launch_large_p<4, 3, 2, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 512) return launch_large_p<8, 2, 1, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 768) return launch_large_p<8, 3, 1, DET, RES, W32>(p, grid_ctas, s);
-    return launch_large_p<8, 4, 1, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 512) return launch_large_p<16, 1, 1, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 640) return launch_large_p<10, 2, 1, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 768) {
+        if constexpr (DET) return launch_large_p<12, 2, 1, DET, RES, W32>(p, grid_ctas, s);
+        else return launch_large_p<8, 3, 1, DET, RES, W32>(p, grid_ctas, s);
+    }
+    if constexpr (DET) return launch_large_p<16, 2, 1, DET, RES, W32>(p, grid_ctas, s);
+    else return launch_large_p<8, 4, 1, DET, RES, W32>(p, grid_ctas, s);
 }
 
-template <int VPT, bool RES, bool W32>
+template <int TPR, int VPT, bool RES, bool W32>
 cudaError_t launch_small_t(const BwdParams& p, cudaStream_t s) {
-    auto kern = bwd_small_kernel<VPT, RES, W32>;
-    const int n_row_ctas = (p.R + kSmallThreads / 32 - 1) / (kSmallThreads / 32);
+    auto kern = bwd_small_kernel<TPR, VPT, RES, W32>;
+    constexpr int RPC = kSmallThreads / TPR;
+    const int n_row_ctas = (p.R + RPC - 1) / RPC;
     const int n_col_ctas = (p.H + kColStrip - 1) / kColStrip;
     const int n_blocks = (p.R + p.block_rows - 1) / p.block_rows;
     const size_t smem = (size_t)n_blocks * kColStrip * sizeof(double);
@@ -756,23 +786,22 @@ cudaError_t launch_small_t(const BwdParams& p, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         smem_set = smem;
     }
-    kern<<<n_row_ctas + n_col_ctas, kSmallThreads, smem, s>>>(p, n_row_ctas);
+    kern<<<n_row_ctas + n_col_ctas, kSmallThreads, smem, s>>>(p);
     return cudaGetLastError();
 }
 
+// Threads per row: one warp up to 256 columns, then up to 256 threads, then more vectors
+// per thread.
 template <bool RES, bool W32>
 cudaError_t dispatch_small(const BwdParams& p, cudaStream_t s) {
-    const int need = (p.nvec + 31) / 32;
-    if (need <= 1) return launch_small_t<1, RES, W32>(p, s);
-    if (need <= 2) return launch_small_t<2, RES, W32>(p, s);
-    if (need <= 4) return launch_small_t<4, RES, W32>(p, s);
-    if (need <= 6) return launch_small_t<6, RES, W32>(p, s);
-    if (need <= 8) return launch_small_t<8, RES, W32>(p, s);
-    if (need <= 12) return launch_small_t<12, RES, W32>(p, s);
-    if (need <= 16) return launch_small_t<16, RES, W32>(p, s);
-    if (need <= 20) return launch_small_t<20, RES, W32>(p, s);
-    if (need <= 24) return launch_small_t<24, RES, W32>(p, s);
-    return launch_small_t<32, RES, W32>(p, s);
+    const int nv = p.nvec;
+    if (nv <= 32) return launch_small_t<32, 1, RES, W32>(p, s);
+    if (nv <= 64) return launch_small_t<64, 1, RES, W32>(p, s);
+    if (nv <= 128) return launch_small_t<128, 1, RES, W32>(p, s);
+    if (nv <= 256) return launch_small_t<256, 1, RES, W32>(p, s);
+    if (nv <= 512) return launch_small_t<256, 2, RES, W32>(p, s);
+    if (nv <= 768) return launch_small_t<256, 3, RES, W32>(p, s);
+    return launch_small_t<256, 4, RES, W32>(p, s);
 }
 
 }  // namespace

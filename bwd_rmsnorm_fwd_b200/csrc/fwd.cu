@@ -315,12 +315,8 @@ __global__ void __launch_bounds__(32 * (1 + SW * L), 1)
             }
             named_bar(1 + slot, ST);
 #pragma unroll
-            for (int q = 0; q < P; ++q) {
-                float a = 0.f;
-#pragma unroll
-                for (int w = 0; w < SW; ++w) a += red[((slot * 2 + buf) * P + q) * SW + w];
-                ss[q] = a;
-            }
+            for (int q = 0; q < P; ++q)
+                ss[q] = warp_sum(lane < SW ? red[((slot * 2 + buf) * P + q) * SW + lane] : 0.f);
             buf ^= 1;
         }
 #pragma unroll
@@ -433,9 +429,9 @@ cudaError_t dispatch_staged(const FwdParams& p, cudaStream_t s) {
     if (nv <= 64) return launch_staged_p<1, 2, 8, RES, W32>(p, s);
     if (nv <= 128) return launch_staged_p<2, 2, 4, RES, W32>(p, s);
     if (nv <= 192) return launch_staged_p<2, 3, 4, RES, W32>(p, s);
-    if (nv <= 256) return launch_staged_p<4, 2, 2, RES, W32>(p, s);
+    if (nv <= 256) return launch_staged_p<2, 4, 4, RES, W32>(p, s);
     if (nv <= 384) return launch_staged_p<4, 3, 2, RES, W32>(p, s);
-    if (nv <= 512) return launch_staged_p<8, 2, 1, RES, W32>(p, s);
+    if (nv <= 512) return launch_staged_p<4, 4, 2, RES, W32>(p, s);
     if (nv <= 768) return launch_staged_p<8, 3, 1, RES, W32>(p, s);
     return launch_staged_p<8, 4, 1, RES, W32>(p, s);
 }

@@ -112,7 +112,8 @@ def test_single_launch_and_pair_give_the_same_bits(T, H):
 
 
 @pytest.mark.parametrize("T,heads,H", [(227, 1, 512), (5000, 1, 1536), (4100, 1, 6144),
-                                       (700, 24, 256), (33000, 1, 264)])
+                                       (700, 24, 256), (33000, 1, 264), (6000, 1, 2048),
+                                       (2500, 1, 4096), (3000, 1, 5120), (2000, 1, 8192)])
 def test_bits_equal_cpu_emulation_of_the_order(T, heads, H):
     x, dy, w, rstd = inputs(T, heads, H, seed=7, family="F3", wdt="fp32")
     B, L, S = api.det_plan(T, heads, H)
