@@ -116,10 +116,17 @@ rmsk::RowsOut out_of(const rms_shape& s, const rms_rows& v) {
 
 // ---- the deterministic order and the program choice --------------------------------------
 
-int32_t det_block_rows(int64_t R) {
+// Rows per block of the deterministic order: 16 in the single-launch regime, otherwise the
+// largest power of two in [8, 64] that still cuts the rows into at least kMinChunks chunks of
+// L blocks (one per SM of a B200), so mid-sized problems keep every SM busy.  A function of
+// (R, L) -- that is, of the row count and the width -- and of nothing else.
+constexpr int64_t kMinChunks = 148;
+
+int32_t det_block_rows(int64_t R, int L) {
     if (R <= 2048) return 16;
-    if (R <= 32768) return 32;
-    return 64;
+    int32_t B = 64;
+    while (B > 8 && (R + (int64_t)B * L - 1) / ((int64_t)B * L) < kMinChunks) B /= 2;
+    return B;
 }
 
 int64_t default_small_rows(int H) {
@@ -141,8 +148,8 @@ struct Plan {
 
 Plan det_plan(int64_t R, int H) {
     Plan p;
-    p.B = det_block_rows(R);
     p.L = rmsk::bwd_slots_for_width(H);
+    p.B = det_block_rows(R, p.L);
     p.S = kFoldSegments;
     const int64_t ch = (int64_t)p.B * p.L;
     p.n_chunks = (int32_t)((R + ch - 1) / ch);

@@ -26,7 +26,7 @@
 //   workspace vector with atomics.  The last CTA to finish (atomic ticket) rounds the
 //   vector to FP32 dw and clears it for the next call.
 //
-// The large kernel gives each CTA L "slots" of SW consumer warps; a slot owns one row at
+// The large kernel gives each CTA L "slots" of ST consumer threads; a slot owns one row at
 // a time and every thread of the slot owns VPT 16-byte column vectors, so the dw state of
 // a column stays in one thread's registers for the whole block.  The per-row dot
 // product is a warp-shuffle tree plus, for multi-warp slots, a named barrier over the
@@ -67,16 +67,20 @@ struct StagedCfg {
     int32_t stage_offset;
 };
 
-template <int SW, int VPT, int L, int P, bool DET, bool RES, bool W32>
-__global__ void __launch_bounds__(32 * (1 + SW * L), 1)
+template <int ST, int VPT, int L, int P, bool DET, bool RES, bool W32>
+__global__ void __launch_bounds__(32 + ST * L, 1)
     bwd_staged_kernel(const BwdParams p, const StagedCfg sc) {
-    constexpr int ST = SW * 32;      // threads per slot
-    constexpr int NCW = SW * L;      // consumer warps
+    // ST threads per slot: a few lanes of a warp (8 or 16: several rows per warp), one warp,
+    // or several warps (a named barrier joins them)
+    static_assert(ST >= 32 ? ST % 32 == 0 : 32 % ST == 0, "slot must tile warps");
+    static_assert((ST * L) % 32 == 0, "consumers must fill whole warps");
+    constexpr int SW = ST >= 32 ? ST / 32 : 1;  // warps per slot
+    constexpr int NCW = ST * L / 32;            // consumer warps
     constexpr int NCT = NCW * 32;    // consumer threads
     constexpr int RT = L * P;        // rows per stage
     constexpr int NTEN = RES ? 3 : 2;
     constexpr int kAllConsumers = 15;  // named barrier over every consumer thread
-    static_assert(16 * kMaxStages + 16 + L * 2 * P * SW * 4 <= kStagedHeader,
+    static_assert(16 * kMaxStages + 16 + (ST > 32 ? L * 2 * P * SW * 4 : 0) <= kStagedHeader,
                   "slot reduction buffers must fit in the header");
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);  // full[kMaxStages], empty[kMaxStages]
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(32 * (1 + SW * L), 1)
                         }
                     }
                 }
-                dot[q] = warp_sum(d2.x + d2.y);
+                dot[q] = group_sum<(ST < 32 ? ST : 32)>(d2.x + d2.y);
             }
             if constexpr (SW > 1) {
                 if (lane == 0) {
@@ -687,10 +691,10 @@ __global__ void __launch_bounds__(kSmallThreads) bwd_small_kernel(const BwdParam
 namespace {
 
 
-template <int SW, int VPT, int L, int P, bool DET, bool RES, bool W32>
+template <int ST, int VPT, int L, int P, bool DET, bool RES, bool W32>
 cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
-    auto kern = bwd_staged_kernel<SW, VPT, L, P, DET, RES, W32>;
-    constexpr int NT = 32 * (1 + SW * L);
+    auto kern = bwd_staged_kernel<ST, VPT, L, P, DET, RES, W32>;
+    constexpr int NT = 32 + ST * L;
     constexpr int NTEN = RES ? 3 : 2;
     constexpr size_t kBudget = 220 * 1024;
     StagedCfg sc;
@@ -738,37 +742,38 @@ cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
 }
 
 // Rows of a slot per stage: 4 when two such stages fit beside the exchange area, else 2.
-template <int SW, int VPT, int L, bool DET, bool RES, bool W32>
+template <int ST, int VPT, int L, bool DET, bool RES, bool W32>
 cudaError_t launch_large_p(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     constexpr size_t kRoom = 220 * 1024 - kStagedHeader;
     const size_t xch = (DET && L > 1) ? (size_t)L * p.nvec * 8 * sizeof(double) : 0;
     const size_t row = (size_t)(RES ? 3 : 2) * L * p.H * 2;
     if (2 * 4 * row + xch + 128 <= kRoom)
-        return launch_large<SW, VPT, L, 4, DET, RES, W32>(p, grid_ctas, s);
-    return launch_large<SW, VPT, L, 2, DET, RES, W32>(p, grid_ctas, s);
+        return launch_large<ST, VPT, L, 4, DET, RES, W32>(p, grid_ctas, s);
+    return launch_large<ST, VPT, L, 2, DET, RES, W32>(p, grid_ctas, s);
 }
 
-// Slot layout per width: SW warps per slot, VPT vectors per thread, L slots per CTA.  L is
-// also the block count of a deterministic chunk and depends on the width only; SW and VPT
-// are free (measured per width and mode): the deterministic mode, which carries a TwoSum
-// state per column, runs best with more warps and fewer columns per thread.
+// Slot layout per width: ST threads per slot, VPT vectors per thread, L slots per CTA.  L is
+// also the block count of a deterministic chunk and depends on the width only (it must match
+// bwd_slots_for_width); ST and VPT are free and were measured per width and mode: narrow rows
+// share a warp between rows, and the deterministic mode, which carries a TwoSum state per
+// column, runs best with more threads and fewer columns per thread.
 template <bool DET, bool RES, bool W32>
 cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     const int nv = p.nvec;
-    if (nv <= 32) return launch_large_p<1, 1, 8, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 64) return launch_large_p<1, 2, 8, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 128) return launch_large_p<2, 2, 4, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 192) return launch_large_p<2, 3, 4, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 256) return launch_large_p<8, 1, 2, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 384) return launch_large_p<4, 3, 2, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 512) return launch_large_p<16, 1, 1, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 640) return launch_large_p<10, 2, 1, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 32) return launch_large_p<16, 2, 16, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 64) return launch_large_p<32, 2, 8, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 128) return launch_large_p<64, 2, 4, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 192) return launch_large_p<96, 2, 4, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 256) return launch_large_p<256, 1, 2, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 384) return launch_large_p<128, 3, 2, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 512) return launch_large_p<512, 1, 1, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 640) return launch_large_p<320, 2, 1, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 768) {
-        if constexpr (DET) return launch_large_p<12, 2, 1, DET, RES, W32>(p, grid_ctas, s);
-        else return launch_large_p<8, 3, 1, DET, RES, W32>(p, grid_ctas, s);
+        if constexpr (DET) return launch_large_p<384, 2, 1, DET, RES, W32>(p, grid_ctas, s);
+        else return launch_large_p<256, 3, 1, DET, RES, W32>(p, grid_ctas, s);
     }
-    if constexpr (DET) return launch_large_p<16, 2, 1, DET, RES, W32>(p, grid_ctas, s);
-    else return launch_large_p<8, 4, 1, DET, RES, W32>(p, grid_ctas, s);
+    if constexpr (DET) return launch_large_p<512, 2, 1, DET, RES, W32>(p, grid_ctas, s);
+    else return launch_large_p<256, 4, 1, DET, RES, W32>(p, grid_ctas, s);
 }
 
 template <int TPR, int VPT, bool RES, bool W32>
@@ -808,6 +813,7 @@ cudaError_t dispatch_small(const BwdParams& p, cudaStream_t s) {
 
 int bwd_slots_for_width(int H) {
     const int nv = H / 8;
+    if (nv <= 32) return 16;
     if (nv <= 64) return 8;
     if (nv <= 192) return 4;
     if (nv <= 384) return 2;

@@ -175,11 +175,16 @@ __device__ __forceinline__ bool rows_contiguous(const RowsIn& v, int32_t heads, 
     return heads == 1 ? v.st == H : (v.sk == H && v.st == (int64_t)heads * H);
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
+// Sum over each group of G consecutive lanes (G a power of two, at most 32); every lane
+// receives its group's sum.
+template <int G>
+__device__ __forceinline__ float group_sum(float v) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
     return v;
 }
+
+__device__ __forceinline__ float warp_sum(float v) { return group_sum<32>(v); }
 
 // TwoSum accumulation of the exact product a*b into (s, c):  p + e == a*b exactly,
 // t + err == s + p exactly; the rounding errors go to the compensation term c.

@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kFwdThreads) fwd_kernel(const FwdParams p) {
 
 // ---- wide rows: bulk-copy pipeline ------------------------------------------------------------
 // Warp 0 streams P rows per slot (x, and the residual in the residual form) into a ring of
-// shared-memory stages with cp.async.bulk; L slots of SW consumer warps each own one row
+// shared-memory stages with cp.async.bulk; L slots of ST consumer threads each own one row
 // at a time: sum of squares (packed FP32 pairs), a shuffle tree plus a named barrier over
 // the slot's warps, then y = (x * rstd) * w stored straight to global memory.  The CTA
 // takes a contiguous row range split evenly between its slots.  Waits are bounded; a wait
@@ -143,14 +143,16 @@ struct FwdStaged {
     int32_t tensor_bytes;
 };
 
-template <int SW, int VPT, int L, int P, bool RES, bool W32>
-__global__ void __launch_bounds__(32 * (1 + SW * L), 1)
+template <int ST, int VPT, int L, int P, bool RES, bool W32>
+__global__ void __launch_bounds__(32 + ST * L, 1)
     fwd_staged_kernel(const FwdParams p, const FwdStaged sc) {
-    constexpr int ST = SW * 32;
-    constexpr int NCW = SW * L;
+    static_assert(ST >= 32 ? ST % 32 == 0 : 32 % ST == 0, "slot must tile warps");
+    static_assert((ST * L) % 32 == 0, "consumers must fill whole warps");
+    constexpr int SW = ST >= 32 ? ST / 32 : 1;  // warps per slot
+    constexpr int NCW = ST * L / 32;
     constexpr int RT = L * P;
     constexpr int NTEN = RES ? 2 : 1;
-    static_assert(16 * kFwdMaxStages + 16 + L * 2 * P * SW * 4 <= kFwdHeader,
+    static_assert(16 * kFwdMaxStages + 16 + (ST > 32 ? L * 2 * P * SW * 4 : 0) <= kFwdHeader,
                   "slot reduction buffers must fit in the header");
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(32 * (1 + SW * L), 1)
                     }
                 }
             }
-            ss[q] = warp_sum(a2.x + a2.y);
+            ss[q] = group_sum<(ST < 32 ? ST : 32)>(a2.x + a2.y);
         }
         if constexpr (SW > 1) {
             if (lane == 0) {
@@ -384,10 +386,10 @@ cudaError_t launch_vpt(const FwdParams& p, bool res, bool w32, cudaStream_t s) {
     return w32 ? launch_one<VPT, 1, false, true>(p, s) : launch_one<VPT, 1, false, false>(p, s);
 }
 
-template <int SW, int VPT, int L, int P, bool RES, bool W32>
+template <int ST, int VPT, int L, int P, bool RES, bool W32>
 cudaError_t launch_staged(const FwdParams& p, cudaStream_t s) {
-    auto kern = fwd_staged_kernel<SW, VPT, L, P, RES, W32>;
-    constexpr int NT = 32 * (1 + SW * L);
+    auto kern = fwd_staged_kernel<ST, VPT, L, P, RES, W32>;
+    constexpr int NT = 32 + ST * L;
     constexpr size_t kBudget = 220 * 1024;
     FwdStaged sc;
     sc.tensor_bytes = L * P * p.H * 2;
@@ -413,27 +415,28 @@ cudaError_t launch_staged(const FwdParams& p, cudaStream_t s) {
 
 // Rows of a slot per stage: the largest of 8, 4, 2 that leaves room for two stages (the
 // larger the tile, the more rows each barrier, reduction and wait is spread over).
-template <int SW, int VPT, int L, bool RES, bool W32>
+template <int ST, int VPT, int L, bool RES, bool W32>
 cudaError_t launch_staged_p(const FwdParams& p, cudaStream_t s) {
     constexpr size_t kRoom = 220 * 1024 - kFwdHeader;
     const size_t row = (size_t)(RES ? 2 : 1) * L * p.H * 2;
-    if (2 * 8 * row <= kRoom) return launch_staged<SW, VPT, L, 8, RES, W32>(p, s);
-    if (2 * 4 * row <= kRoom) return launch_staged<SW, VPT, L, 4, RES, W32>(p, s);
-    return launch_staged<SW, VPT, L, 2, RES, W32>(p, s);
+    if (2 * 8 * row <= kRoom) return launch_staged<ST, VPT, L, 8, RES, W32>(p, s);
+    if (2 * 4 * row <= kRoom) return launch_staged<ST, VPT, L, 4, RES, W32>(p, s);
+    return launch_staged<ST, VPT, L, 2, RES, W32>(p, s);
 }
 
 template <bool RES, bool W32>
 cudaError_t dispatch_staged(const FwdParams& p, cudaStream_t s) {
+    // ST threads per slot (narrow rows share a warp), VPT vectors per thread, L slots
     const int nv = p.nvec;
-    if (nv <= 32) return launch_staged_p<1, 1, 8, RES, W32>(p, s);
-    if (nv <= 64) return launch_staged_p<1, 2, 8, RES, W32>(p, s);
-    if (nv <= 128) return launch_staged_p<2, 2, 4, RES, W32>(p, s);
-    if (nv <= 192) return launch_staged_p<2, 3, 4, RES, W32>(p, s);
-    if (nv <= 256) return launch_staged_p<2, 4, 4, RES, W32>(p, s);
-    if (nv <= 384) return launch_staged_p<4, 3, 2, RES, W32>(p, s);
-    if (nv <= 512) return launch_staged_p<4, 4, 2, RES, W32>(p, s);
-    if (nv <= 768) return launch_staged_p<8, 3, 1, RES, W32>(p, s);
-    return launch_staged_p<8, 4, 1, RES, W32>(p, s);
+    if (nv <= 32) return launch_staged_p<16, 2, 16, RES, W32>(p, s);
+    if (nv <= 64) return launch_staged_p<32, 2, 8, RES, W32>(p, s);
+    if (nv <= 128) return launch_staged_p<64, 2, 4, RES, W32>(p, s);
+    if (nv <= 192) return launch_staged_p<64, 3, 4, RES, W32>(p, s);
+    if (nv <= 256) return launch_staged_p<64, 4, 4, RES, W32>(p, s);
+    if (nv <= 384) return launch_staged_p<128, 3, 2, RES, W32>(p, s);
+    if (nv <= 512) return launch_staged_p<128, 4, 2, RES, W32>(p, s);
+    if (nv <= 768) return launch_staged_p<256, 3, 1, RES, W32>(p, s);
+    return launch_staged_p<256, 4, 1, RES, W32>(p, s);
 }
 
 }  // namespace
