@@ -213,6 +213,19 @@ def run_reference(args):
     return 0
 
 
+# ---- multi-rank plumbing ----------------------------------------------------------------------
+
+def max_over_ranks(value, dist, device):
+    """The maximum of `value` over all ranks (the step time of a replica job is that of its
+    slowest rank); `dist` is torch.distributed or None for one process."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---- GPU timing helpers ----------------------------------------------------------------------
 
 def make_inputs(T, H, wdt, seed, device, torch):
@@ -427,11 +440,7 @@ def main():
     api.status(ws)
     step_us = [a.elapsed_time(c) * 1e3 for a, b, c in evs]
     bwd_us = [b.elapsed_time(c) * 1e3 for a, b, c in evs]
-    ms_step = sum(step_us) / len(step_us) / 1e3
-    if dist:
-        t = torch.tensor([ms_step], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = max_over_ranks(sum(step_us) / len(step_us) / 1e3, dist, dev)
     us_step = ms_step * 1e3
     bwd_avg_us = sum(bwd_us) / len(bwd_us)
     step_bytes = 2 * bytes_fwd(R, H, wb) + bytes_bwd(R, H, wb)

@@ -150,9 +150,6 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
         // ================= producer =================
         int j = 0;
         for (int u = 0; u < n_units; ++u) {
-            int base[L], endr[L];
-#pragma unroll
-            for (int s = 0; s < L; ++s) { base[s] = slot_base(u, s); endr[s] = slot_end(u, s); }
             const int nt = unit_tiles(u);
             for (int t = 0; t < nt; ++t, ++j) {
                 const int stage = j % NS;
@@ -166,10 +163,10 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                 if (*abort_flag) goto drain;
                 uint32_t bytes = 0;
 #pragma unroll
-                for (int s = 0; s < L; ++s)
-#pragma unroll
-                    for (int q = 0; q < P; ++q)
-                        if (base[s] + t * P + q < endr[s]) bytes += row_bytes * NTEN;
+                for (int s = 0; s < L; ++s) {
+                    const int n = min(P, slot_end(u, s) - (slot_base(u, s) + t * P));
+                    if (n > 0) bytes += (uint32_t)n * row_bytes * NTEN;
+                }
                 if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), bytes);
                 __syncwarp();
                 const uint32_t sbase = smem_addr(stages + (size_t)stage * sc.stage_bytes);
@@ -179,8 +176,8 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                     const int s = c - ten * L;
                     const RowsIn& src = ten == 0 ? p.x : (ten == 1 ? p.dy : p.dh);
                     if (!rows_contiguous(src, p.heads, H)) continue;
-                    const int row0 = base[s] + t * P;
-                    const int n = min(P, endr[s] - row0);
+                    const int row0 = slot_base(u, s) + t * P;
+                    const int n = min(P, slot_end(u, s) - row0);
                     if (n > 0)
                         bulk_load(sbase + (uint32_t)ten * sc.tensor_bytes +
                                       (uint32_t)(s * P) * row_bytes,
@@ -192,9 +189,9 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                     const int rr = c - ten * RT;
                     const int s = rr / P;
                     const int q = rr - s * P;
-                    const int row = base[s] + t * P + q;
+                    const int row = slot_base(u, s) + t * P + q;
                     const RowsIn& src = ten == 0 ? p.x : (ten == 1 ? p.dy : p.dh);
-                    if (row < endr[s] && !rows_contiguous(src, p.heads, H)) {
+                    if (row < slot_end(u, s) && !rows_contiguous(src, p.heads, H)) {
                         bulk_load(sbase + (uint32_t)ten * sc.tensor_bytes + (uint32_t)rr * row_bytes,
                                   src.ptr + row_offset(row, p.heads, src.st, src.sk), row_bytes,
                                   full_bar(stage));
@@ -767,7 +764,7 @@ cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     if (nv <= 256) return launch_large_p<256, 1, 2, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 384) return launch_large_p<128, 3, 2, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 512) return launch_large_p<512, 1, 1, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 640) return launch_large_p<320, 2, 1, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 640) return launch_large_p<640, 1, 1, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 768) {
         if constexpr (DET) return launch_large_p<384, 2, 1, DET, RES, W32>(p, grid_ctas, s);
         else return launch_large_p<256, 3, 1, DET, RES, W32>(p, grid_ctas, s);

@@ -186,9 +186,6 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
     const int nt = (maxlen + P - 1) / P;
 
     if (warp == 0) {
-        int base[L], endr[L];
-#pragma unroll
-        for (int s = 0; s < L; ++s) { base[s] = sbase(s); endr[s] = sbase(s + 1); }
         int j = 0;
         for (; j < nt; ++j) {
             const int stage = j % NS;
@@ -200,10 +197,10 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
             if (*abort_flag) break;
             uint32_t bytes = 0;
 #pragma unroll
-            for (int s = 0; s < L; ++s)
-#pragma unroll
-                for (int q = 0; q < P; ++q)
-                    if (base[s] + j * P + q < endr[s]) bytes += row_bytes * NTEN;
+            for (int s = 0; s < L; ++s) {
+                const int n = min(P, sbase(s + 1) - (sbase(s) + j * P));
+                if (n > 0) bytes += (uint32_t)n * row_bytes * NTEN;
+            }
             if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), bytes);
             __syncwarp();
             const uint32_t sb = smem_addr(stages + (size_t)stage * sc.stage_bytes);
@@ -213,8 +210,8 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                 const int s = c - ten * L;
                 const RowsIn& src = ten == 0 ? p.x : p.res;
                 if (!rows_contiguous(src, p.heads, H)) continue;
-                const int row0 = base[s] + j * P;
-                const int n = min(P, endr[s] - row0);
+                const int row0 = sbase(s) + j * P;
+                const int n = min(P, sbase(s + 1) - row0);
                 if (n > 0)
                     bulk_load(sb + (uint32_t)ten * sc.tensor_bytes + (uint32_t)(s * P) * row_bytes,
                               src.ptr + row_offset(row0, p.heads, src.st, src.sk),
@@ -225,9 +222,9 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                 const int rr = c - ten * RT;
                 const int s = rr / P;
                 const int q = rr - s * P;
-                const int row = base[s] + j * P + q;
+                const int row = sbase(s) + j * P + q;
                 const RowsIn& src = ten == 0 ? p.x : p.res;
-                if (row < endr[s] && !rows_contiguous(src, p.heads, H)) {
+                if (row < sbase(s + 1) && !rows_contiguous(src, p.heads, H)) {
                     bulk_load(sb + (uint32_t)ten * sc.tensor_bytes + (uint32_t)rr * row_bytes,
                               src.ptr + row_offset(row, p.heads, src.st, src.sk), row_bytes,
                               full_bar(stage));
@@ -435,6 +432,7 @@ cudaError_t dispatch_staged(const FwdParams& p, cudaStream_t s) {
     if (nv <= 256) return launch_staged_p<64, 4, 4, RES, W32>(p, s);
     if (nv <= 384) return launch_staged_p<128, 3, 2, RES, W32>(p, s);
     if (nv <= 512) return launch_staged_p<128, 4, 2, RES, W32>(p, s);
+    if (nv <= 640) return launch_staged_p<128, 5, 2, RES, W32>(p, s);
     if (nv <= 768) return launch_staged_p<256, 3, 1, RES, W32>(p, s);
     return launch_staged_p<256, 4, 1, RES, W32>(p, s);
 }
