@@ -18,7 +18,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "librmsnorm_train.so")
 
-SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "noalloc.cu", "tma.cu"]
 HEADERS = [os.path.join(CSRC, "common.cuh"), os.path.join(INCLUDE, "rmsnorm_train.h")]
 
 NVCC_FLAGS = [

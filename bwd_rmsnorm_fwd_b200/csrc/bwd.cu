@@ -69,7 +69,7 @@ struct StagedCfg {
 
 template <int ST, int VPT, int L, int P, bool DET, bool RES, bool W32>
 __global__ void __launch_bounds__(32 + ST * L, 1)
-    bwd_staged_kernel(const BwdParams p, const StagedCfg sc) {
+    bwd_staged_kernel(const BwdParams p, const StagedCfg sc, const __grid_constant__ RowMaps tm) {
     // ST threads per slot: a few lanes of a warp (8 or 16: several rows per warp), one warp,
     // or several warps (a named barrier joins them)
     static_assert(ST >= 32 ? ST % 32 == 0 : 32 % ST == 0, "slot must tile warps");
@@ -148,6 +148,9 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
 
     if (warp == 0) {
         // ================= producer =================
+        // tensor loads also need a 128-byte aligned destination (checked once, used for both
+        // the byte count and the copies)
+        const bool tma_ok = (smem_addr(stages) & 127u) == 0 && (row_bytes & 127u) == 0;
         int j = 0;
         for (int u = 0; u < n_units; ++u) {
             const int nt = unit_tiles(u);
@@ -161,27 +164,33 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                 }
                 __syncwarp();
                 if (*abort_flag) goto drain;
-                uint32_t bytes = 0;
+                uint32_t bytes = 0;  // a TMA box always lands whole (rows past the end as 0)
 #pragma unroll
                 for (int s = 0; s < L; ++s) {
                     const int n = min(P, slot_end(u, s) - (slot_base(u, s) + t * P));
-                    if (n > 0) bytes += (uint32_t)n * row_bytes * NTEN;
+                    if (n > 0)
+#pragma unroll
+                        for (int ten = 0; ten < NTEN; ++ten)
+                            bytes += (uint32_t)(tm.use[ten] && tma_ok ? P : n) * row_bytes;
                 }
                 if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), bytes);
                 __syncwarp();
                 const uint32_t sbase = smem_addr(stages + (size_t)stage * sc.stage_bytes);
-                // one copy per (tensor, slot) when rows are contiguous, else one per row
+                // one TMA box per (tensor, slot) for equally spaced rows of H <= 256, one bulk
+                // copy per (tensor, slot) for contiguous rows, else one bulk copy per row
                 for (int c = lane; c < L * NTEN; c += 32) {
                     const int ten = c / L;
                     const int s = c - ten * L;
                     const RowsIn& src = ten == 0 ? p.x : (ten == 1 ? p.dy : p.dh);
-                    if (!rows_contiguous(src, p.heads, H)) continue;
                     const int row0 = slot_base(u, s) + t * P;
                     const int n = min(P, slot_end(u, s) - row0);
-                    if (n > 0)
-                        bulk_load(sbase + (uint32_t)ten * sc.tensor_bytes +
-                                      (uint32_t)(s * P) * row_bytes,
-                                  src.ptr + row_offset(row0, p.heads, src.st, src.sk),
+                    if (n <= 0) continue;
+                    const uint32_t dst =
+                        sbase + (uint32_t)ten * sc.tensor_bytes + (uint32_t)(s * P) * row_bytes;
+                    if (tm.use[ten] && tma_ok)
+                        tma_load_rows(dst, &tm.map[ten], row0, full_bar(stage));
+                    else if (rows_contiguous(src, p.heads, H))
+                        bulk_load(dst, src.ptr + row_offset(row0, p.heads, src.st, src.sk),
                                   (uint32_t)n * row_bytes, full_bar(stage));
                 }
                 for (int c = lane; c < RT * NTEN; c += 32) {
@@ -191,7 +200,7 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                     const int q = rr - s * P;
                     const int row = slot_base(u, s) + t * P + q;
                     const RowsIn& src = ten == 0 ? p.x : (ten == 1 ? p.dy : p.dh);
-                    if (row < slot_end(u, s) && !rows_contiguous(src, p.heads, H)) {
+                    if (row < slot_end(u, s) && !(tm.use[ten] && tma_ok) && !rows_contiguous(src, p.heads, H)) {
                         bulk_load(sbase + (uint32_t)ten * sc.tensor_bytes + (uint32_t)rr * row_bytes,
                                   src.ptr + row_offset(row, p.heads, src.st, src.sk), row_bytes,
                                   full_bar(stage));
@@ -721,7 +730,10 @@ cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
         if (need < 1) need = 1;
         grid = (int)(need < cap ? need : cap);
     }
-    kern<<<grid, NT, smem, s>>>(p, sc);
+    RowMaps tm;
+    const RowsIn views[3] = {p.x, p.dy, p.dh};
+    make_row_maps(&tm, views, RES ? 3 : 2, p.heads, p.H, p.R, P);
+    kern<<<grid, NT, smem, s>>>(p, sc, tm);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || !DET) return e;
     // fold kernel, programmatic dependent launch

@@ -1,6 +1,7 @@
 // Internal declarations shared by the kernels and the C-ABI layer of librmsnorm_train.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap and its enums (types only; the encoder is fetched at run time)
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -57,6 +58,13 @@ struct BwdParams {
     int64_t wait_cycles;
 };
 
+// TMA descriptors of up to three row tensors (x / dy / dh, or x / residual); use[i] != 0
+// when tensor i has equally spaced rows of H <= 256 and its descriptor is valid.
+struct alignas(64) RowMaps {
+    CUtensorMap map[3];
+    int32_t use[3];
+};
+
 // device status bits
 constexpr unsigned kStatusTimeout = 1u;
 // default limit of a device-side wait (about two seconds at 2 GHz)
@@ -75,6 +83,10 @@ cudaError_t launch_bwd_nondet(const BwdParams& p, bool residual, bool w32, int g
 // (the blocks of one deterministic chunk).  Also the chunk's block count.
 int bwd_slots_for_width(int H);
 int device_sm_count();
+// Fills `maps` for the first n views (box of box_rows rows x H); tensors that cannot use a
+// descriptor get use = 0 and keep the bulk-copy path.
+void make_row_maps(RowMaps* maps, const RowsIn* views, int n, int heads, int H, int64_t rows,
+                   int box_rows);
 // Reads and clears the forward's device status word (a library global on the current
 // device); synchronises `s` first.
 cudaError_t fwd_status_take(cudaStream_t s, unsigned* word);
@@ -164,6 +176,7 @@ __device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16x2(v.x, v.
 __device__ __forceinline__ int64_t row_offset(int32_t r, int32_t heads, int64_t st,
                                               int64_t sk) {
     if (heads == 1) return (int64_t)r * st;
+    if (st == (int64_t)heads * sk) return (int64_t)r * sk;  // equally spaced rows: no division
     const int32_t t = r / heads;
     const int32_t k = r - t * heads;
     return (int64_t)t * st + (int64_t)k * sk;
@@ -260,6 +273,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
         if (mbar_test(bar, parity)) return true;
         if (clock64() - t0 > limit) return false;
     }
+}
+
+// 2-D tiled TMA load of rows [row0, row0 + box rows) of a row tensor (box = H x rows) into
+// shared memory, completion counted on `bar`.  x is always 0 (16-byte aligned); rows past
+// the tensor's end are filled with zeros and still counted.
+__device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap* map, int row0,
+                                              uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row0), "r"(bar)
+        : "memory");
 }
 
 // Bulk copy global -> shared (this CTA), completion counted in bytes on `bar`.

@@ -145,7 +145,7 @@ struct FwdStaged {
 
 template <int ST, int VPT, int L, int P, bool RES, bool W32>
 __global__ void __launch_bounds__(32 + ST * L, 1)
-    fwd_staged_kernel(const FwdParams p, const FwdStaged sc) {
+    fwd_staged_kernel(const FwdParams p, const FwdStaged sc, const __grid_constant__ RowMaps tm) {
     static_assert(ST >= 32 ? ST % 32 == 0 : 32 % ST == 0, "slot must tile warps");
     static_assert((ST * L) % 32 == 0, "consumers must fill whole warps");
     constexpr int SW = ST >= 32 ? ST / 32 : 1;  // warps per slot
@@ -186,6 +186,9 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
     const int nt = (maxlen + P - 1) / P;
 
     if (warp == 0) {
+        // tensor loads also need a 128-byte aligned destination (checked once, used for both
+        // the byte count and the copies)
+        const bool tma_ok = (smem_addr(stages) & 127u) == 0 && (row_bytes & 127u) == 0;
         int j = 0;
         for (; j < nt; ++j) {
             const int stage = j % NS;
@@ -195,26 +198,33 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
             }
             __syncwarp();
             if (*abort_flag) break;
-            uint32_t bytes = 0;
+            uint32_t bytes = 0;  // a TMA box always lands whole (rows past the end as 0)
 #pragma unroll
             for (int s = 0; s < L; ++s) {
                 const int n = min(P, sbase(s + 1) - (sbase(s) + j * P));
-                if (n > 0) bytes += (uint32_t)n * row_bytes * NTEN;
+                if (n > 0)
+#pragma unroll
+                    for (int ten = 0; ten < NTEN; ++ten)
+                        bytes += (uint32_t)(tm.use[ten] && tma_ok ? P : n) * row_bytes;
             }
             if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), bytes);
             __syncwarp();
             const uint32_t sb = smem_addr(stages + (size_t)stage * sc.stage_bytes);
-            // one copy per (tensor, slot) when rows are contiguous, else one per row
+            // one TMA box per (tensor, slot) for equally spaced rows of H <= 256, one bulk copy
+            // per (tensor, slot) for contiguous rows, else one bulk copy per row
             for (int c = lane; c < L * NTEN; c += 32) {
                 const int ten = c / L;
                 const int s = c - ten * L;
                 const RowsIn& src = ten == 0 ? p.x : p.res;
-                if (!rows_contiguous(src, p.heads, H)) continue;
                 const int row0 = sbase(s) + j * P;
                 const int n = min(P, sbase(s + 1) - row0);
-                if (n > 0)
-                    bulk_load(sb + (uint32_t)ten * sc.tensor_bytes + (uint32_t)(s * P) * row_bytes,
-                              src.ptr + row_offset(row0, p.heads, src.st, src.sk),
+                if (n <= 0) continue;
+                const uint32_t dst =
+                    sb + (uint32_t)ten * sc.tensor_bytes + (uint32_t)(s * P) * row_bytes;
+                if (tm.use[ten] && tma_ok)
+                    tma_load_rows(dst, &tm.map[ten], row0, full_bar(stage));
+                else if (rows_contiguous(src, p.heads, H))
+                    bulk_load(dst, src.ptr + row_offset(row0, p.heads, src.st, src.sk),
                               (uint32_t)n * row_bytes, full_bar(stage));
             }
             for (int c = lane; c < RT * NTEN; c += 32) {
@@ -224,7 +234,7 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                 const int q = rr - s * P;
                 const int row = sbase(s) + j * P + q;
                 const RowsIn& src = ten == 0 ? p.x : p.res;
-                if (row < sbase(s + 1) && !rows_contiguous(src, p.heads, H)) {
+                if (row < sbase(s + 1) && !(tm.use[ten] && tma_ok) && !rows_contiguous(src, p.heads, H)) {
                     bulk_load(sb + (uint32_t)ten * sc.tensor_bytes + (uint32_t)rr * row_bytes,
                               src.ptr + row_offset(row, p.heads, src.st, src.sk), row_bytes,
                               full_bar(stage));
@@ -406,7 +416,10 @@ cudaError_t launch_staged(const FwdParams& p, cudaStream_t s) {
     int64_t need = ((int64_t)p.R + L * 4 - 1) / (L * 4);
     const int64_t cap = device_sm_count();
     const int grid = (int)(need < cap ? need : cap);
-    kern<<<grid, NT, smem, s>>>(p, sc);
+    RowMaps tm;
+    const RowsIn views[2] = {p.x, p.res};
+    make_row_maps(&tm, views, RES ? 2 : 1, p.heads, p.H, p.R, P);
+    kern<<<grid, NT, smem, s>>>(p, sc, tm);
     return cudaGetLastError();
 }
 
