@@ -539,10 +539,11 @@ __global__ void __launch_bounds__(32 * kFoldSegMax) bwd_fold_kernel(const BwdPar
 
 constexpr int kSmallThreads = 512;
 constexpr int kColStrip = 64;   // columns per column task
-constexpr int kRowBatch = 16;   // rows loaded together by a column-task lane
+constexpr int kRowBatch = 8;    // rows loaded together by a column-task lane (short code:
+                                 // with a cold L2 the instructions come from DRAM too)
 
 template <int TPR, int VPT, bool RES, bool W32>
-__global__ void __launch_bounds__(kSmallThreads) bwd_small_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(kSmallThreads, 2) bwd_small_kernel(const BwdParams p) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int H = p.H;
