@@ -123,6 +123,86 @@ __global__ void __launch_bounds__(kFwdThreads) fwd_kernel(const FwdParams p) {
     }
 }
 
+// ---- few wide rows: one CTA per row -----------------------------------------------------------
+// Below a pipeline's worth of rows per SM, a row wider than 4 vectors per lane is spread over
+// the warps of one CTA (thread t holds vectors t, t + NT, ...; at most 4 of them), so R rows
+// occupy R SMs instead of R/8, and the code stays short: after an L2 flush its first fetch is
+// part of the call's latency.  The warp sums meet in shared memory and every thread adds them
+// in warp order (two buffers, one barrier per row).
+constexpr int kFwdRowMaxThreads = 256;
+
+template <int VPT, bool RES, bool W32>
+__global__ void __launch_bounds__(kFwdRowMaxThreads) fwd_row_cta_kernel(const FwdParams p) {
+    __shared__ float red[2][kFwdRowMaxThreads / 32];
+    const int nt = (int)blockDim.x;
+    const int nw = nt >> 5;
+    const int t = (int)threadIdx.x;
+    const float invH = 1.0f / (float)p.H;
+    int buf = 0;
+    for (int r = blockIdx.x; r < p.R; r += gridDim.x, buf ^= 1) {
+        const int64_t ox = row_offset(r, p.heads, p.x.st, p.x.sk);
+        uint4 xv[VPT];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int v = t + nt * i;
+            xv[i] = v < p.nvec ? ld_stream16(p.x.ptr + ox + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        if constexpr (RES) {
+            const int64_t orr = row_offset(r, p.heads, p.res.st, p.res.sk);
+            const int64_t oh = row_offset(r, p.heads, p.h.st, p.h.sk);
+            uint4 rv4[VPT];
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int v = t + nt * i;
+                rv4[i] = v < p.nvec ? ld_stream16(p.res.ptr + orr + 8 * v)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                float a[8], b[8];
+                unpack8(xv[i], a);
+                unpack8(rv4[i], b);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) a[e] = __fadd_rn(a[e], b[e]);
+                xv[i] = pack8(a);  // h = BF16(x + res): the norm runs on rounded h
+                const int v = t + nt * i;
+                if (v < p.nvec) st16(p.h.ptr + oh + 8 * v, xv[i]);
+            }
+        }
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            float f[8];
+            unpack8(xv[i], f);
+            const float s01 = __fadd_rn(__fmul_rn(f[0], f[0]), __fmul_rn(f[1], f[1]));
+            const float s23 = __fadd_rn(__fmul_rn(f[2], f[2]), __fmul_rn(f[3], f[3]));
+            const float s45 = __fadd_rn(__fmul_rn(f[4], f[4]), __fmul_rn(f[5], f[5]));
+            const float s67 = __fadd_rn(__fmul_rn(f[6], f[6]), __fmul_rn(f[7], f[7]));
+            acc = __fadd_rn(acc, __fadd_rn(__fadd_rn(s01, s23), __fadd_rn(s45, s67)));
+        }
+        acc = warp_sum(acc);
+        if ((t & 31) == 0) red[buf][t >> 5] = acc;
+        __syncthreads();
+        float ss = red[buf][0];
+        for (int k = 1; k < nw; ++k) ss = __fadd_rn(ss, red[buf][k]);
+        const float rs = rsqrtf(__fmaf_rn(ss, invH, p.eps));
+        const int64_t oy = row_offset(r, p.heads, p.y.st, p.y.sk);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int v = t + nt * i;
+            if (v < p.nvec) {
+                float f[8], wf[8];
+                unpack8(xv[i], f);
+                load_w8<W32>(p.w, 8 * v, wf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], rs), wf[e]);
+                st16(p.y.ptr + oy + 8 * v, pack8(f));
+            }
+        }
+        if (t == 0) p.rstd[r] = rs;
+    }
+}
+
 // ---- wide rows: bulk-copy pipeline ------------------------------------------------------------
 // Warp 0 streams P rows per slot (x, and the residual in the residual form) into a ring of
 // shared-memory stages with cp.async.bulk; L slots of ST consumer threads each own one row
@@ -393,6 +473,26 @@ cudaError_t launch_vpt(const FwdParams& p, bool res, bool w32, cudaStream_t s) {
     return w32 ? launch_one<VPT, 1, false, true>(p, s) : launch_one<VPT, 1, false, false>(p, s);
 }
 
+// One CTA per row, 4 vectors per thread: ceil(nvec / 128) warps (2..8 for H in (1024, 8192]).
+template <bool RES, bool W32>
+cudaError_t launch_row_cta(const FwdParams& p, cudaStream_t s) {
+    constexpr int kVpt = 4;
+    auto kern = fwd_row_cta_kernel<kVpt, RES, W32>;
+    const int warps = (p.nvec + 32 * kVpt - 1) / (32 * kVpt);
+    if (warps * 32 > kFwdRowMaxThreads) return cudaErrorInvalidConfiguration;
+    static int occ[kFwdRowMaxThreads / 32 + 1] = {};  // resident CTAs per SM, by warp count
+    if (occ[warps] == 0) {
+        int o = 0;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, warps * 32, 0);
+        if (e != cudaSuccess) return e;
+        occ[warps] = o > 0 ? o : 1;
+    }
+    const int64_t cap = (int64_t)device_sm_count() * occ[warps];
+    const int grid = (int)(p.R < cap ? p.R : cap);
+    kern<<<grid, warps * 32, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
 template <int ST, int VPT, int L, int P, bool RES, bool W32>
 cudaError_t launch_staged(const FwdParams& p, cudaStream_t s) {
     auto kern = fwd_staged_kernel<ST, VPT, L, P, RES, W32>;
@@ -470,19 +570,13 @@ cudaError_t launch_fwd(const FwdParams& p, bool res, bool w32, cudaStream_t s) {
         if (res) return w32 ? dispatch_staged<true, true>(p, s) : dispatch_staged<true, false>(p, s);
         return w32 ? dispatch_staged<false, true>(p, s) : dispatch_staged<false, false>(p, s);
     }
-    const int need = (p.nvec + 31) / 32;  // vectors per lane
+    const int need = (p.nvec + 31) / 32;  // vectors per lane of a warp-wide row
     if (need <= 1) return launch_vpt<1, 4>(p, res, w32, s);
     if (need <= 2) return launch_vpt<2, 2>(p, res, w32, s);
     if (need <= 3) return launch_vpt<3, 1>(p, res, w32, s);
     if (need <= 4) return launch_vpt<4, 1>(p, res, w32, s);
-    if (need <= 6) return launch_vpt<6, 1>(p, res, w32, s);
-    if (need <= 8) return launch_vpt<8, 1>(p, res, w32, s);
-    if (need <= 12) return launch_vpt<12, 1>(p, res, w32, s);
-    if (need <= 16) return launch_vpt<16, 1>(p, res, w32, s);
-    if (need <= 20) return launch_vpt<20, 1>(p, res, w32, s);
-    if (need <= 24) return launch_vpt<24, 1>(p, res, w32, s);
-    if (need <= 28) return launch_vpt<28, 1>(p, res, w32, s);
-    return launch_vpt<32, 1>(p, res, w32, s);
+    if (res) return w32 ? launch_row_cta<true, true>(p, s) : launch_row_cta<true, false>(p, s);
+    return w32 ? launch_row_cta<false, true>(p, s) : launch_row_cta<false, false>(p, s);
 }
 
 }  // namespace rmsk
