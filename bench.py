@@ -11,8 +11,8 @@ for this step on B200 (flashinfer PR #8848 table, H6144 T131072, BF16 weight).
 Every launch inside the timed region is one of librmsnorm_train's kernels.  The JSON
 line also carries the roofline of the dominant kernel (the backward), the CPU oracle
 as a baseline, an end-to-end figure with host buffers, SM clocks sampled during the
-timed region, and a per-configuration table (CUDA-graph replay, cold L2) with the
-achieved fraction of the measured HBM bandwidth.
+timed region, and a per-configuration table (CUPTI span of a CUDA-graph replay, cold L2,
+the pages' timing rule) with the achieved fraction of the measured HBM bandwidth.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
        [--sweep all|none]
@@ -294,44 +294,95 @@ def kernel_time_us(fn, flush, torch, reps=30):
     return total / reps
 
 
+def call_spans_us(events, flush_tag="FillFunctor"):
+    """Per-call spans from device records (name, start_us, end_us) of a loop that flushes L2
+    before every call: records sorted by start, cut at every flush kernel; a call's span runs
+    from its first record's start to its last record's end."""
+    spans, lo, hi = [], None, None
+    for name, start, end in sorted(events, key=lambda e: e[1]):
+        if flush_tag in name:
+            if lo is not None:
+                spans.append(hi - lo)
+            lo = hi = None
+        else:
+            lo = start if lo is None else min(lo, start)
+            hi = end if hi is None else max(hi, end)
+    if lo is not None:
+        spans.append(hi - lo)
+    return spans
+
+
+def span_time_us(fn, flush, torch, reps=30):
+    """Median CUPTI span of one call replayed from a CUDA graph with L2 flushed before each
+    replay (the pages' timing rule): first kernel start to last kernel end, every kernel of
+    the call inside the span."""
+    from torch.autograd import DeviceType
+    from torch.profiler import ProfilerActivity, profile
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    try:
+        with torch.cuda.graph(g):
+            fn()
+        run = g.replay
+    except Exception:
+        run = fn
+    run()
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        for _ in range(reps):
+            flush.zero_()
+            run()
+        torch.cuda.synchronize()
+    events = [(e.name, e.time_range.start, e.time_range.end) for e in prof.events()
+              if e.device_type == DeviceType.CUDA]
+    del g
+    spans = call_spans_us(events)
+    if not spans:
+        raise RuntimeError("the profiler recorded no device activity for the call")
+    return statistics.median(spans)
+
+
 SWEEP_GROUPS = ("tiny", "small-T", "residual", "per-head", "large-T")
 
 
 def sweep(torch, api, flush, peak, dev, groups=SWEEP_GROUPS):
-    """Per-configuration table: us per call (graph replay, cold L2) and fraction of the
-    measured HBM bandwidth, for every BASELINE configuration."""
+    """Per-configuration table: us per call (CUPTI span of a graph replay, cold L2; CUDA events
+    around the replay too where a call is long enough) and the fraction of the measured HBM
+    bandwidth, for every configuration of the pages' tables."""
     out = []
     ws = api.Workspace(dev)
 
-    def rec(cfg, form, H, T, wdt, op, us, nbytes, timer_name):
+    def rec(cfg, form, H, T, wdt, op, fn, nbytes, replay):
+        us = span_time_us(fn, flush, torch)
         gbs = nbytes / (us * 1e-6) / 1e9
-        out.append({"cfg": cfg, "form": form, "H": H, "T": T, "w": wdt, "op": op,
-                    "us": round(us, 2), "gbs": round(gbs, 1), "frac": round(gbs / peak, 3),
-                    "timer": timer_name})
+        row = {"cfg": cfg, "form": form, "H": H, "T": T, "w": wdt, "op": op,
+               "us": round(us, 2), "gbs": round(gbs, 1), "frac": round(gbs / peak, 3),
+               "timer": "cupti_span"}
+        if replay:
+            row["replay_us"] = round(graph_time_us(fn, flush, torch), 2)
+        out.append(row)
 
     def ops(cfg, form, x, dy, w, H, T, R, wdt, heads=1, res=None, dh=None, do=("fwd", "det", "nondet")):
         wb = 2 if wdt == "bf16" else 4
         isres = res is not None
-        # a few microseconds per call: CUPTI kernel time; otherwise graph replay
-        small = R * H <= (1 << 22)
-        tname = "cupti_kernel" if small else "graph_replay"
-        timer = ((lambda fn: kernel_time_us(fn, flush, torch)) if small else
-                 (lambda fn: graph_time_us(fn, flush, torch)))
+        # CUDA events around a graph replay as well, where a call outlasts the launch latency
+        replay = R * H > (1 << 22)
         if isres:
             h, _, rstd = api.rmsnorm_train_fwd(x, w, residual=res)
         else:
             _, rstd = api.rmsnorm_train_fwd(x, w)
             h = x
         if "fwd" in do:
-            us = timer(lambda: api.rmsnorm_train_fwd(x, w, residual=res))
-            rec(cfg, form, H, T, wdt, "fwd", us, bytes_fwd(R, H, wb, isres), tname)
+            rec(cfg, form, H, T, wdt, "fwd", lambda: api.rmsnorm_train_fwd(x, w, residual=res),
+                bytes_fwd(R, H, wb, isres), replay)
         for det in (True, False):
             if ("det" if det else "nondet") not in do:
                 continue
-            us = timer(lambda: api.rmsnorm_train_bwd(h, w, rstd, dy, deterministic=det, dh=dh,
-                                                     workspace=ws))
-            rec(cfg, form, H, T, wdt, "bwd_det" if det else "bwd_nondet", us,
-                bytes_bwd(R, H, wb, isres), tname)
+            rec(cfg, form, H, T, wdt, "bwd_det" if det else "bwd_nondet",
+                lambda: api.rmsnorm_train_bwd(h, w, rstd, dy, deterministic=det, dh=dh,
+                                              workspace=ws),
+                bytes_bwd(R, H, wb, isres), replay)
 
     # Tiny and small-T sweep (deterministic backward, single launch)
     if "tiny" in groups:

@@ -158,6 +158,6 @@ def status(workspace: Workspace | None = None, device=None) -> None:
 
 
 def forward_status() -> None:
-    """Raises RmsError if a forward on the current device recorded a device-side error;
-    clears the word."""
+    """Synchronises the current stream and raises RmsError on a CUDA error there (the
+    forward kernels have no device-side waits and no status word of their own)."""
     _lib.check(_lib.lib().rms_status(None, _stream()))

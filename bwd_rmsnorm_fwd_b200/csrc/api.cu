@@ -304,7 +304,6 @@ int rms_train_fwd(rms_shape shape, rms_rows x, const void* w, int w_dtype, rms_r
     p.w = w;
     p.rstd = rstd;
     p.eps = eps;
-    p.wait_cycles = g_wait_cycles;
     cudaError_t e = rmsk::launch_fwd(p, false, w_dtype == RMS_FP32, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "forward launch");
 }
@@ -341,7 +340,6 @@ int rms_residual_train_fwd(rms_shape shape, rms_rows x, rms_rows residual, const
     p.w = w;
     p.rstd = rstd;
     p.eps = eps;
-    p.wait_cycles = g_wait_cycles;
     cudaError_t e = rmsk::launch_fwd(p, true, w_dtype == RMS_FP32, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "residual forward launch");
 }
@@ -403,8 +401,10 @@ int rms_status(void* workspace, void* stream) {
     unsigned word = 0;
     cudaError_t e;
     if (!workspace) {
-        e = rmsk::fwd_status_take(st, &word);
-        if (e != cudaSuccess) return cuda_fail(e, "reading the forward status word");
+        // the forward kernels take no workspace and have no device-side waits: only the
+        // stream's own errors can be reported
+        e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
     } else {
         e = cudaStreamSynchronize(st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");

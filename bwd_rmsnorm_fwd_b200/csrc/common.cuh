@@ -29,7 +29,6 @@ struct FwdParams {
     const void* w;
     float* rstd;
     float eps;
-    int64_t wait_cycles;  // limit of every device-side wait, in SM clock cycles
 };
 
 struct BwdParams {
@@ -89,7 +88,6 @@ void make_row_maps(RowMaps* maps, const RowsIn* views, int n, int heads, int H, 
                    int box_rows);
 // Reads and clears the forward's device status word (a library global on the current
 // device); synchronises `s` first.
-cudaError_t fwd_status_take(cudaStream_t s, unsigned* word);
 // Records `msg` as this thread's rms_last_error() text and returns `code`.
 int set_error(int code, const char* msg);
 

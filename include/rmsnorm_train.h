@@ -156,17 +156,18 @@ int rms_train_bwd_path(rms_shape shape, int deterministic);
 int64_t rms_set_small_rows_limit(int64_t rows);
 
 /* Limit, in SM clock cycles, of every device-side wait of later launches in this
- * process (the bulk-copy pipelines' barrier waits); the default is about two seconds.  A
- * wait that reaches it makes the kernel record RMS_ETIMEOUT in its status word (see
- * rms_status) and finish without waiting further; its outputs are then invalid.  Shorter limits exist to test that path (0 makes every wait a single
- * non-blocking probe); a negative value restores the default.  Returns the previous
- * limit.  Not thread-safe against concurrent launches. */
+ * process (the backward's bulk-copy pipeline barrier waits; the forward has none); the
+ * default is about two seconds.  A wait that reaches it makes the kernel record
+ * RMS_ETIMEOUT in its workspace status word (see rms_status) and finish without waiting
+ * further; its outputs are then invalid.  Shorter limits exist to test that path (0
+ * makes every wait a single non-blocking probe); a negative value restores the default.
+ * Returns the previous limit.  Not thread-safe against concurrent launches. */
 int64_t rms_set_wait_limit_cycles(int64_t cycles);
 
-/* Synchronises `stream`, reads and clears the device status word of `workspace` (the
- * backward's), or, with workspace == NULL, the forward's status word (one per device,
- * inside the library: the forward takes no workspace).  Returns RMS_OK, RMS_ETIMEOUT or
- * RMS_ECUDA. */
+/* Synchronises `stream` and reads and clears the device status word of `workspace`
+ * (written by the backward).  With workspace == NULL it only synchronises: the forward
+ * takes no workspace and has no device-side waits, so the stream's own errors are all
+ * there is to report.  Returns RMS_OK, RMS_ETIMEOUT or RMS_ECUDA. */
 int rms_status(void* workspace, void* stream);
 
 /* Message for the last non-zero return on this thread ("" if none). */

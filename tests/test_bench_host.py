@@ -79,3 +79,15 @@ def test_algorithmic_bytes():
     assert bench.bytes_bwd(R, H, 4) == 6 * R * H + 4 * H + 4 * R + 4 * H
     assert bench.bytes_fwd(R, H, 2, res=True) == 8 * R * H + 2 * H + 4 * R
     assert bench.bytes_bwd(R, H, 2, res=True) == 8 * R * H + 2 * H + 4 * R + 4 * H
+
+
+def test_call_spans_cut_at_the_flush_kernel():
+    """Spans run from a call's first record to its last one; every flush closes a call, and
+    overlapping records (a dependent launch that starts before its producer ends) count once."""
+    fill = "at::vectorized_elementwise_kernel<4, at::FillFunctor<float>>"
+    ev = [(fill, 0.0, 50.0), ("rmsk::main", 51.0, 60.0), ("rmsk::fold", 59.0, 63.5),
+          (fill, 70.0, 120.0), ("rmsk::one", 121.0, 125.0),
+          (fill, 130.0, 180.0)]
+    assert bench.call_spans_us(list(reversed(ev))) == [12.5, 4.0]
+    assert bench.call_spans_us([(fill, 0.0, 1.0)]) == []
+    assert bench.call_spans_us([("rmsk::k", 2.0, 5.0)]) == [3.0]

@@ -46,27 +46,20 @@ def test_wait_limit_reports_timeout_and_context_survives(det):
         assert_dw(dw.cpu().numpy(), dw_ref, f"after timeout det={det}")
 
 
-def test_forward_wait_limit_reports_timeout():
-    """The forward's pipeline waits are bounded too; with no workspace its status word is
-    the library's own, read through rms_status(NULL)."""
+def test_forward_has_no_waits_to_time_out():
+    """The forward kernels never wait on the device: with the wait limit at zero cycles the
+    forward still completes, correct, and its status check stays clean."""
     T, H = 32768, 6144
     x = synth.rows(14, "x", T, H)
     w = synth.weight(14, H, "fp32")
     y_ref, rstd_ref = oracle.train_fwd(x, w)
     xd, wd = dev_rows(x), dev_weight(w)
     L = _lib.lib()
-    api.forward_status()
     prev = L.rms_set_wait_limit_cycles(0)
     try:
-        api.rmsnorm_train_fwd(xd, wd)
-        torch.cuda.synchronize()
+        y, rstd = api.rmsnorm_train_fwd(xd, wd)
+        api.forward_status()
     finally:
         L.rms_set_wait_limit_cycles(prev)
-    with pytest.raises(_lib.RmsError) as ei:
-        api.forward_status()
-    assert ei.value.code == _lib.RMS_ETIMEOUT
-    api.forward_status()
-    y, rstd = api.rmsnorm_train_fwd(xd, wd)
-    api.forward_status()
     from gpu_common import assert_fwd, host_bits
-    assert_fwd(host_bits(y), rstd.cpu().numpy(), y_ref, rstd_ref, "forward after timeout")
+    assert_fwd(host_bits(y), rstd.cpu().numpy(), y_ref, rstd_ref, "forward at wait limit 0")

@@ -117,9 +117,9 @@ def test_large_widths_ragged_rows(H, wdt):
 @pytest.mark.parametrize("residual", [False, True])
 @pytest.mark.parametrize("H,T", [(1032, 2367), (1536, 148), (6144, 5), (8192, 2000)])
 def test_few_wide_rows(H, T, residual):
-    """Row counts below the pipelined forward's cut-over (16 rows per SM) at widths above
-    four vectors per lane, where a row is spread over the warps of one CTA; ragged widths
-    and a padded row stride."""
+    """Widths above four vectors per lane, where the forward spreads a row over the warps of
+    one CTA: ragged widths (H 1032: one thread holds a single vector), a padded row stride,
+    and row counts from a handful to a few per resident CTA."""
     run_case(T, 1, H, "fp32" if H % 3 == 0 else "bf16", seed=H + T, residual=residual,
              layout=(H + 64, H))
 
