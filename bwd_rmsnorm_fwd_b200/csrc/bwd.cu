@@ -14,16 +14,15 @@
 //   FP64.  Chunk partials are cut into S contiguous segments, each folded left to
 //   right, and the segment sums are folded left to right and rounded once to FP32.
 //   B, L and S depend only on the row count and H, so the bits never depend on the
-//   grid or on the SM count.  Three programs produce exactly these bits:
+//   grid or on the SM count.  Two programs produce exactly these bits:
 //     - bwd_small_kernel: one launch; row tasks compute dx, column tasks walk every
 //       row of a 64-column strip and do the whole fold (used for small row counts);
 //     - bwd_staged_kernel<DET> + bwd_fold_kernel: CTAs take whole chunks (each slot of
 //       the CTA one block), write FP64 chunk partials to the workspace, and the fold
 //       kernel (launched with programmatic dependent launch) finishes the order.
-// * non-deterministic: each CTA takes a contiguous row range; every thread sums eight
-//   rows at a time in FP32 (one FMA per element), adds each eight-row block into an
-//   FP64 accumulator in shared memory, and the CTA adds its totals into an FP64
-//   workspace vector with atomics.  The last CTA to finish (atomic ticket) rounds the
+// * non-deterministic: every thread sums eight rows at a time in FP32 (one FMA per
+//   element) and adds each eight-row block into FP64 registers; a CTA's totals meet in
+//   shared memory and the CTA adds them into an FP64 workspace vector with atomics.  The last CTA to finish (atomic ticket) rounds the
 //   vector to FP32 dw and clears it for the next call.
 //
 // The large kernel gives each CTA L "slots" of ST consumer threads; a slot owns one row at
@@ -490,6 +489,219 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
 }
 
 // ============================================================================================
+// Narrow-row kernel for mid-sized blocked-FP32 backwards (H <= 512, R*H < 2^24): one warp per
+// row, no producer warp and no barrier on the data path.  Lane l owns the column vectors l and
+// l + 32 of every row, so its dw state never leaves registers.  Each warp runs its own
+// S-stage ring in shared memory, filled with per-lane cp.async: lane l copies its own 16-byte
+// vectors of x, dy (and dh) and the row's rstd S-1 rows ahead and later reads back only what
+// it copied itself, so a per-thread cp.async.wait_group is all the synchronisation the ring
+// needs.  With no pipeline to fill and drain per CTA it finishes small problems sooner than
+// the bulk-copy kernel; on large ones it issues about 1.8x the instructions per row (a lane
+// holds only 8 or 16 elements of a row) and the bulk-copy kernel is faster, so it is used
+// below 2^24 elements only.  Rows are taken grid-stride; eight-row FP32 blocks go into FP64
+// registers; the warp totals meet in shared memory, then one FP64 atomic per column per CTA
+// and the last-CTA ticket, as in the bulk-copy kernel.
+// ============================================================================================
+
+constexpr int kWarpBwdWarps = 8;
+constexpr int64_t kWarpBwdMaxElems = int64_t(1) << 24;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Bytes of one ring stage of one warp: NTEN tensors x VPT vectors x 32 lanes x 16 bytes, then
+// 32 lanes x 4 bytes of rstd.
+template <int VPT, bool RES>
+__host__ __device__ constexpr int warp_stage_bytes() {
+    return (RES ? 3 : 2) * VPT * 32 * 16 + 32 * 4;
+}
+
+template <int VPT, int S, bool RES, bool W32>
+__global__ void __launch_bounds__(32 * kWarpBwdWarps) bwd_warp_kernel(const BwdParams p) {
+    constexpr int NTEN = RES ? 3 : 2;
+    constexpr int SB = warp_stage_bytes<VPT, RES>();
+    constexpr int nw = kWarpBwdWarps;
+    extern __shared__ __align__(16) unsigned char wsmem[];
+    __shared__ unsigned last;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int H = p.H;
+    const int nvec = p.nvec;
+    const float invH = 1.0f / (float)H;
+    double* tot = reinterpret_cast<double*>(wsmem);  // [warps][H]
+    unsigned char* ring = wsmem + (size_t)nw * H * sizeof(double) + (size_t)warp * S * SB;
+    const uint32_t ring_s = smem_addr(ring);
+
+    float2 w2[VPT][4];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int v = lane + 32 * i;
+        float wf[8];
+        if (v < nvec) {
+            load_w8<W32>(p.w, 8 * v, wf);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) wf[e] = 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w2[i][k] = make_float2(wf[2 * k], wf[2 * k + 1]);
+    }
+    // s = eight-row FP32 block of -dw, acc = FP64 total of dw
+    float2 s2[VPT][4];
+    double acc[VPT][8];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) s2[i][k] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[i][e] = 0.0;
+    }
+
+    // the warp's rows: gw, gw + (warps in the grid), ...
+    const int gw = blockIdx.x * nw + warp;
+    const int nwt = gridDim.x * nw;
+    const int total = p.R > gw ? (p.R - 1 - gw) / nwt + 1 : 0;
+    auto issue = [&](int j) {
+        if (j < total) {
+            const int r = gw + j * nwt;
+            const uint32_t st = ring_s + (uint32_t)((j % S) * SB);
+            const int64_t ox = row_offset(r, p.heads, p.x.st, p.x.sk);
+            const int64_t od = row_offset(r, p.heads, p.dy.st, p.dy.sk);
+            const int64_t oh = RES ? row_offset(r, p.heads, p.dh.st, p.dh.sk) : 0;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int v = lane + 32 * i;
+                if (v < nvec) {
+                    cp_async16(st + (uint32_t)((0 * VPT + i) * 512 + lane * 16), p.x.ptr + ox + 8 * v);
+                    cp_async16(st + (uint32_t)((1 * VPT + i) * 512 + lane * 16), p.dy.ptr + od + 8 * v);
+                    if constexpr (RES)
+                        cp_async16(st + (uint32_t)((2 * VPT + i) * 512 + lane * 16), p.dh.ptr + oh + 8 * v);
+                }
+            }
+            cp_async4(st + (uint32_t)(NTEN * VPT * 512 + lane * 4), p.rstd + r);
+        }
+        cp_async_commit();  // one group per row, empty or not: wait_group counts them
+    };
+
+#pragma unroll
+    for (int j = 0; j < S - 1; ++j) issue(j);
+    int in_block = 0;
+    for (int j = 0; j < total; ++j) {
+        cp_async_wait<S - 2>();  // this lane's copies of row j have landed
+        const int r = gw + j * nwt;
+        const unsigned char* st = ring + (j % S) * SB;
+        const float rs = *reinterpret_cast<const float*>(st + NTEN * VPT * 512 + lane * 4);
+        uint4 xv[VPT], dv[VPT], hv[RES ? VPT : 1];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int v = lane + 32 * i;
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            xv[i] = v < nvec ? *reinterpret_cast<const uint4*>(st + (0 * VPT + i) * 512 + lane * 16) : z;
+            dv[i] = v < nvec ? *reinterpret_cast<const uint4*>(st + (1 * VPT + i) * 512 + lane * 16) : z;
+            if constexpr (RES)
+                hv[i] = v < nvec ? *reinterpret_cast<const uint4*>(st + (2 * VPT + i) * 512 + lane * 16) : z;
+        }
+        // pass 1: the row's sum of g * (-xh)
+        const float2 nrs = make_float2(-rs, -rs);
+        float2 d2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+            const uint32_t dw4[4] = {dv[i].x, dv[i].y, dv[i].z, dv[i].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 nx = mul2(bf16x2_to_f2(xw[k]), nrs);
+                const float2 gg = mul2(bf16x2_to_f2(dw4[k]), w2[i][k]);
+                d2 = fma2(gg, nx, d2);
+            }
+        }
+        const float dot = warp_sum(d2.x + d2.y);
+        // pass 2: dx = rstd (g + nx c), c = -dot / H; the row's dw terms
+        const float cr = -dot * invH;
+        const float2 c2v = make_float2(cr, cr);
+        const float2 rs2 = make_float2(rs, rs);
+        uint16_t* dxrow = p.dx.ptr + row_offset(r, p.heads, p.dx.st, p.dx.sk);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int v = lane + 32 * i;
+            if (v >= nvec) continue;
+            const uint32_t xw[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+            const uint32_t dw4[4] = {dv[i].x, dv[i].y, dv[i].z, dv[i].w};
+            uint32_t hw[4] = {0u, 0u, 0u, 0u};
+            if constexpr (RES) {
+                hw[0] = hv[i].x; hw[1] = hv[i].y; hw[2] = hv[i].z; hw[3] = hv[i].w;
+            }
+            uint32_t out[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 d = bf16x2_to_f2(dw4[k]);
+                const float2 nx = mul2(bf16x2_to_f2(xw[k]), nrs);
+                const float2 gg = mul2(d, w2[i][k]);
+                float2 o = mul2(fma2(nx, c2v, gg), rs2);
+                if constexpr (RES) o = add2(o, bf16x2_to_f2(hw[k]));
+                out[k] = pack2(o);
+                s2[i][k] = fma2(d, nx, s2[i][k]);
+            }
+            st16(dxrow + 8 * v, make_uint4(out[0], out[1], out[2], out[3]));
+        }
+        if (++in_block == 8) {  // eight-row FP32 blocks go into the FP64 total
+#pragma unroll
+            for (int i = 0; i < VPT; ++i)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    acc[i][2 * k] -= (double)s2[i][k].x;
+                    acc[i][2 * k + 1] -= (double)s2[i][k].y;
+                    s2[i][k] = make_float2(0.f, 0.f);
+                }
+            in_block = 0;
+        }
+        issue(j + S - 1);
+    }
+    cp_async_wait<0>();
+
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int v = lane + 32 * i;
+        if (v >= nvec) continue;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            tot[(size_t)warp * H + 8 * v + 2 * k] = acc[i][2 * k] - (double)s2[i][k].x;
+            tot[(size_t)warp * H + 8 * v + 2 * k + 1] = acc[i][2 * k + 1] - (double)s2[i][k].y;
+        }
+    }
+    __syncthreads();
+    for (int col = threadIdx.x; col < H; col += blockDim.x) {
+        double a = tot[col];
+        for (int b = 1; b < nw; ++b) a += tot[(size_t)b * H + col];
+        atomicAdd(p.acc + col, a);
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = (atomicAdd(p.ticket, 1u) == gridDim.x - 1) ? 1u : 0u;
+    __syncthreads();
+    if (last) {
+        __threadfence();
+        for (int col = threadIdx.x; col < H; col += blockDim.x) {
+            const double a = __ldcg(p.acc + col);
+            p.dw[col] = __double2float_rn(a);
+            p.acc[col] = 0.0;
+        }
+        if (threadIdx.x == 0) *p.ticket = 0u;
+    }
+}
+
+// ============================================================================================
 // Fold kernel: chunk partials -> dw, in the fixed segment order.
 // ============================================================================================
 
@@ -698,6 +910,8 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bwd_small_kernel(const BwdPa
 namespace {
 
 
+cudaError_t launch_fold(const BwdParams& p, cudaStream_t s);
+
 template <int ST, int VPT, int L, int P, bool DET, bool RES, bool W32>
 cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     auto kern = bwd_staged_kernel<ST, VPT, L, P, DET, RES, W32>;
@@ -737,7 +951,49 @@ cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     kern<<<grid, NT, smem, s>>>(p, sc, tm);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || !DET) return e;
-    // fold kernel, programmatic dependent launch
+    return launch_fold(p, s);
+}
+
+// Mid-sized blocked-FP32 backward of narrow rows: one warp per row, VPT vectors per lane, an
+// S-stage cp.async ring per warp, 8-warp CTAs.
+template <int VPT, int S, bool RES, bool W32>
+cudaError_t launch_warp_bwd(const BwdParams& p, int grid_ctas, cudaStream_t s) {
+    auto kern = bwd_warp_kernel<VPT, S, RES, W32>;
+    constexpr int nw = kWarpBwdWarps;
+    if (p.nvec > 32 * VPT) return cudaErrorInvalidConfiguration;
+    const size_t ring = (size_t)nw * S * warp_stage_bytes<VPT, RES>();
+    const size_t smem = (size_t)nw * p.H * sizeof(double) + ring;
+    const size_t smem_max = (size_t)nw * 256 * VPT * sizeof(double) + ring;  // widest row
+    static int occ = 0;  // resident CTAs per SM at the widest row of this instantiation
+    if (occ == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem_max);
+        if (e != cudaSuccess) return e;
+        int o = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, nw * 32, smem_max);
+        if (e != cudaSuccess) return e;
+        occ = o > 0 ? o : 1;
+    }
+    int grid = grid_ctas;
+    if (grid <= 0) {
+        int64_t need = ((int64_t)p.R + nw - 1) / nw;
+        if (need < 1) need = 1;
+        const int64_t cap = (int64_t)device_sm_count() * occ;
+        grid = (int)(need < cap ? need : cap);
+    }
+    kern<<<grid, nw * 32, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <bool RES, bool W32>
+cudaError_t dispatch_warp_bwd(const BwdParams& p, int grid_ctas, cudaStream_t s) {
+    constexpr int S = RES ? 6 : 8;
+    if (p.nvec <= 32) return launch_warp_bwd<1, S, RES, W32>(p, grid_ctas, s);
+    return launch_warp_bwd<2, S, RES, W32>(p, grid_ctas, s);
+}
+
+// fold kernel after a deterministic main kernel, programmatic dependent launch
+cudaError_t launch_fold(const BwdParams& p, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((p.H + 31) / 32));
     cfg.blockDim = dim3(32 * kFoldSegMax);
@@ -770,6 +1026,10 @@ cudaError_t launch_large_p(const BwdParams& p, int grid_ctas, cudaStream_t s) {
 template <bool DET, bool RES, bool W32>
 cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     const int nv = p.nvec;
+    if constexpr (!DET) {
+        if (nv <= 64 && (int64_t)p.R * p.H < kWarpBwdMaxElems)
+            return dispatch_warp_bwd<RES, W32>(p, grid_ctas, s);
+    }
     if (nv <= 32) return launch_large_p<16, 2, 16, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 64) return launch_large_p<32, 2, 8, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 128) return launch_large_p<64, 2, 4, DET, RES, W32>(p, grid_ctas, s);

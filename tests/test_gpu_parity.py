@@ -124,6 +124,16 @@ def test_few_wide_rows(H, T, residual):
              layout=(H + 64, H))
 
 
+@pytest.mark.parametrize("residual", [False, True])
+@pytest.mark.parametrize("H,T,grid", [(256, 20000, 0), (264, 9001, 1), (512, 12000, 1000),
+                                      (256, 5000, 7)])
+def test_blocked_fp32_narrow_rows(H, T, residual, grid):
+    """The blocked-FP32 backward of narrow rows below 2^24 elements (one warp per row, a
+    cp.async ring per warp): plain and residual forms, a ragged width, and grids from one
+    CTA (every warp walks many rows) to more CTAs than rows per warp."""
+    run_case(T, 1, H, "bf16", seed=H + T, residual=residual, modes=(False,), grid_ctas=grid)
+
+
 # ---- edge cases ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("H", [8, 24, 264, 776, 8192])
