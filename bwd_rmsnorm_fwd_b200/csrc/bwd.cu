@@ -847,8 +847,11 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bwd_small_kernel(const BwdPa
     const bool jok = j < H;
     const int B = p.block_rows;
     const int n_blocks = (p.R + B - 1) / B;
+    const float2 m1 = make_float2(-1.f, -1.f);
     for (int b = warp; b < n_blocks; b += kSmallThreads / 32) {
-        float s0 = 0.f, k0 = 0.f, s1 = 0.f, k1 = 0.f;
+        // TwoSum state (sum, compensation) of the lane's two columns, as packed pairs: every
+        // packed operation rounds each lane like the scalar one, and the code is half as long
+        float2 s2 = make_float2(0.f, 0.f), k2 = make_float2(0.f, 0.f);
         const int rb0 = b * B;
         const int rb1 = min(rb0 + B, p.R);
         for (int r = rb0; r < rb1; r += kRowBatch) {
@@ -869,13 +872,21 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bwd_small_kernel(const BwdPa
             for (int u = 0; u < kRowBatch; ++u) {
                 const float rs = __shfl_sync(0xFFFFFFFFu, rsl, u);
                 if (r + u < rb1) {
-                    twosum_product(bf16lo(dw2[u]), __fmul_rn(bf16lo(xw[u]), rs), s0, k0);
-                    twosum_product(bf16hi(dw2[u]), __fmul_rn(bf16hi(xw[u]), rs), s1, k1);
+                    // exact product p + e == dy * xh, then TwoSum of (s, p), per column
+                    const float2 d = bf16x2_to_f2(dw2[u]);
+                    const float2 xh = mul2(bf16x2_to_f2(xw[u]), make_float2(rs, rs));
+                    const float2 pp = mul2(d, xh);
+                    const float2 e = fma2(d, xh, mul2(pp, m1));
+                    const float2 tt = add2(s2, pp);
+                    const float2 z = sub2(tt, s2);
+                    const float2 err = add2(sub2(s2, sub2(tt, z)), sub2(pp, z));
+                    k2 = add2(k2, add2(err, e));
+                    s2 = tt;
                 }
             }
         }
-        bp[(size_t)b * kColStrip + 2 * lane] = (double)s0 + (double)k0;
-        bp[(size_t)b * kColStrip + 2 * lane + 1] = (double)s1 + (double)k1;
+        bp[(size_t)b * kColStrip + 2 * lane] = (double)s2.x + (double)k2.x;
+        bp[(size_t)b * kColStrip + 2 * lane + 1] = (double)s2.y + (double)k2.y;
     }
     __syncthreads();
     const int t = threadIdx.x;

@@ -197,20 +197,6 @@ __device__ __forceinline__ float group_sum(float v) {
 
 __device__ __forceinline__ float warp_sum(float v) { return group_sum<32>(v); }
 
-// TwoSum accumulation of the exact product a*b into (s, c):  p + e == a*b exactly,
-// t + err == s + p exactly; the rounding errors go to the compensation term c.
-// Written with explicit round-to-nearest intrinsics so nothing is contracted or
-// reassociated: the deterministic order depends on this exact sequence.
-__device__ __forceinline__ void twosum_product(float a, float b, float& s, float& c) {
-    const float p = __fmul_rn(a, b);
-    const float e = __fmaf_rn(a, b, -p);
-    const float t = __fadd_rn(s, p);
-    const float z = __fsub_rn(t, s);
-    const float err = __fadd_rn(__fsub_rn(s, __fsub_rn(t, z)), __fsub_rn(p, z));
-    c = __fadd_rn(c, __fadd_rn(err, e));
-    s = t;
-}
-
 // ---- shared-memory barriers and bulk copies (sm_90+ PTX) -----------------------------------
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
