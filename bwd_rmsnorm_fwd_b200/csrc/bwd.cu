@@ -506,20 +506,6 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
 constexpr int kWarpBwdWarps = 8;
 constexpr int64_t kWarpBwdMaxElems = int64_t(1) << 24;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // Bytes of one ring stage of one warp: NTEN tensors x VPT vectors x 32 lanes x 16 bytes, then
 // 32 lanes x 4 bytes of rstd.
 template <int VPT, bool RES>

@@ -197,6 +197,21 @@ __device__ __forceinline__ float group_sum(float v) {
 
 __device__ __forceinline__ float warp_sum(float v) { return group_sum<32>(v); }
 
+// ---- per-thread asynchronous copies (cp.async): a thread waits for its own copies only -------
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ---- shared-memory barriers and bulk copies (sm_90+ PTX) -----------------------------------
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {

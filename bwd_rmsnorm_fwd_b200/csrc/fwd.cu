@@ -5,7 +5,7 @@
 // (flashinfer PR #8848 introduction and "Workload"; PR #8512 "Residual rows".)
 //
 // Design: every row is read from HBM once into registers, reduced, scaled and written
-// back; nothing is staged in shared memory.  The forward reads a row once and writes it
+// back.  The forward reads a row once and writes it
 // once, so what sets its speed is how many bytes are in flight per SM and how little
 // work sits between a row's last load and its first store.  Many small resident CTAs with
 // all of a row's loads issued before any use beat a shared-memory pipeline with one CTA
@@ -16,7 +16,8 @@
 //     group of ROWS rows for the narrowest widths once there are rows enough to fill the
 //     GPU), a 5-level shuffle tree per row;
 //   * wider rows: one CTA per row, every thread VPT vectors of it (2 up to H 4096, 4
-//     above), warp sums met in shared memory.
+//     above), warp sums met in shared memory; in the residual form at H > 4096 and many
+//     rows, the rows pass through a two-row per-thread cp.async ring in shared memory.
 //
 // Both grids are persistent (SM count x resident CTAs) and walk rows in order, which keeps
 // neighbouring CTAs on neighbouring DRAM pages.  Squares of BF16 values are exact in FP32;
@@ -143,10 +144,13 @@ __global__ void __launch_bounds__(kFwdWarpThreads) fwd_warp_kernel(const FwdPara
 
 // ---- wider rows: one CTA per row ----------------------------------------------------------------
 // Thread t holds vectors t, t + NT, ... (VPT of them) of the row, so a warp's loads and stores
-// are whole 512-byte runs.  With PF the next row's vectors are loaded before the current row
-// is reduced and written, which keeps loads in flight through the reduction and the stores.
-// The warp sums meet in shared memory and every thread adds them in warp order (two buffers,
-// one barrier per row).
+// are whole 512-byte runs.  The warp sums meet in shared memory and every thread adds them in
+// warp order (two buffers, one barrier per row).  With D >= 2 the rows pass through a ring of D
+// rows in shared memory filled by per-thread cp.async: thread t copies its own vectors of the
+// CTA's next D-1 rows before it reduces and writes the current one, and reads back only what it
+// copied itself, so its own cp.async.wait_group is all the synchronisation the ring needs and the
+// loads stay in flight through the reduction, the barrier and the stores at no register cost.
+// D == 0 loads each row straight into registers.
 constexpr int kFwdRowMaxThreads = 256;
 
 template <int VPT, bool RES>
@@ -170,21 +174,54 @@ __device__ __forceinline__ void load_row(const FwdParams& p, int r, uint4 (&xv)[
     }
 }
 
-template <int VPT, bool PF, bool RES, bool W32>
+template <int VPT, int D, bool RES, bool W32>
 __global__ void __launch_bounds__(kFwdRowMaxThreads) fwd_row_cta_kernel(const FwdParams p) {
+    constexpr int NTEN = RES ? 2 : 1;
     __shared__ float red[2][kFwdRowMaxThreads / 32];
+    extern __shared__ __align__(16) uint4 ring[];  // [D][NTEN][VPT][NT] 16-byte vectors
     const int nt = (int)blockDim.x;
     const int nw = nt >> 5;
     const int t = (int)threadIdx.x;
     const float invH = 1.0f / (float)p.H;
-    uint4 xv[VPT], rv[RES ? VPT : 1];
-    int r = blockIdx.x;
-    if (PF && r < p.R) load_row<VPT, RES>(p, r, xv, rv);
-    for (int buf = 0; r < p.R; r += gridDim.x, buf ^= 1) {
-        if constexpr (!PF) load_row<VPT, RES>(p, r, xv, rv);
-        uint4 xn[PF ? VPT : 1], rn[PF && RES ? VPT : 1];
-        if constexpr (PF) {
-            if (r + (int)gridDim.x < p.R) load_row<VPT, RES>(p, r + gridDim.x, xn, rn);
+    const int G = (int)gridDim.x;
+    auto slot = [&](int k, int ten, int i) -> uint4* {
+        return ring + (((k % (D > 0 ? D : 1)) * NTEN + ten) * VPT + i) * nt + t;
+    };
+    // D >= 2: copies of the k-th row of this CTA (row blockIdx.x + k*G), one group per row
+    auto issue = [&](int k) {
+        const int r = (int)blockIdx.x + k * G;
+        if (r < p.R) {
+            const int64_t ox = row_offset(r, p.heads, p.x.st, p.x.sk);
+            const int64_t orr = RES ? row_offset(r, p.heads, p.res.st, p.res.sk) : 0;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int v = t + nt * i;
+                if (v < p.nvec) {
+                    cp_async16(smem_addr(slot(k, 0, i)), p.x.ptr + ox + 8 * v);
+                    if constexpr (RES) cp_async16(smem_addr(slot(k, 1, i)), p.res.ptr + orr + 8 * v);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+    if constexpr (D >= 2) {
+#pragma unroll
+        for (int k = 0; k < D - 1; ++k) issue(k);
+    }
+    int buf = 0;
+    for (int k = 0, r = blockIdx.x; r < p.R; ++k, r += G, buf ^= 1) {
+        uint4 xv[VPT], rv[RES ? VPT : 1];
+        if constexpr (D >= 2) {
+            issue(k + D - 1);
+            cp_async_wait<D - 1>();  // this thread's copies of row k have landed
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const bool in = t + nt * i < p.nvec;
+                xv[i] = in ? *slot(k, 0, i) : make_uint4(0u, 0u, 0u, 0u);
+                if constexpr (RES) rv[i] = in ? *slot(k, 1, i) : make_uint4(0u, 0u, 0u, 0u);
+            }
+        } else {
+            load_row<VPT, RES>(p, r, xv, rv);
         }
         if constexpr (RES) {
             const int64_t oh = row_offset(r, p.heads, p.h.st, p.h.sk);
@@ -202,7 +239,7 @@ __global__ void __launch_bounds__(kFwdRowMaxThreads) fwd_row_cta_kernel(const Fw
         if ((t & 31) == 0) red[buf][t >> 5] = acc;
         __syncthreads();
         float ss = red[buf][0];
-        for (int k = 1; k < nw; ++k) ss = __fadd_rn(ss, red[buf][k]);
+        for (int q = 1; q < nw; ++q) ss = __fadd_rn(ss, red[buf][q]);
         const float rs = rsqrtf(__fmaf_rn(ss, invH, p.eps));
         const int64_t oy = row_offset(r, p.heads, p.y.st, p.y.sk);
 #pragma unroll
@@ -211,24 +248,18 @@ __global__ void __launch_bounds__(kFwdRowMaxThreads) fwd_row_cta_kernel(const Fw
             if (v < p.nvec) st16(p.y.ptr + oy + 8 * v, scale8<W32>(xv[i], rs, p.w, v));
         }
         if (t == 0) p.rstd[r] = rs;
-        if constexpr (PF) {
-#pragma unroll
-            for (int i = 0; i < VPT; ++i) {
-                xv[i] = xn[i];
-                if constexpr (RES) rv[i] = rn[i];
-            }
-        }
     }
+    if constexpr (D >= 2) cp_async_wait<0>();
 }
 
 namespace {
 
 // Resident CTAs per SM of a kernel at a block size (cached per kernel and block size).
 template <typename K>
-int resident_ctas(K kern, int threads, int* cache) {
+int resident_ctas(K kern, int threads, int* cache, size_t smem = 0) {
     if (*cache == 0) {
         int o = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, threads, 0) != cudaSuccess)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, threads, smem) != cudaSuccess)
             return -1;
         *cache = o > 0 ? o : 1;
     }
@@ -266,30 +297,43 @@ cudaError_t launch_warp_vpt(const FwdParams& p, bool res, bool w32, cudaStream_t
     return w32 ? launch_warp<VPT, 1, false, true>(p, s) : launch_warp<VPT, 1, false, false>(p, s);
 }
 
-// One CTA per row: ceil(nvec / (32 VPT)) warps.
-template <int VPT, bool PF, bool RES, bool W32>
+// One CTA per row: ceil(nvec / (32 VPT)) warps; a D-row cp.async ring when D >= 2.
+template <int VPT, int D, bool RES, bool W32>
 cudaError_t launch_row_cta(const FwdParams& p, cudaStream_t s) {
-    auto kern = fwd_row_cta_kernel<VPT, PF, RES, W32>;
+    auto kern = fwd_row_cta_kernel<VPT, D, RES, W32>;
     const int warps = (p.nvec + 32 * VPT - 1) / (32 * VPT);
     if (warps * 32 > kFwdRowMaxThreads) return cudaErrorInvalidConfiguration;
+    const size_t smem = D >= 2 ? (size_t)D * (RES ? 2 : 1) * VPT * warps * 32 * 16 : 0;
+    if constexpr (D >= 2) {
+        // the ring of the widest row this instantiation serves (above the 48 KB default)
+        static bool attr = false;
+        if (!attr) {
+            const int most = D * (RES ? 2 : 1) * VPT * kFwdRowMaxThreads * 16;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+            if (e != cudaSuccess) return e;
+            attr = true;
+        }
+    }
     static int occ[kFwdRowMaxThreads / 32 + 1] = {};  // by warp count
-    const int o = resident_ctas(kern, warps * 32, &occ[warps]);
+    const int o = resident_ctas(kern, warps * 32, &occ[warps], smem);
     if (o < 0) return cudaGetLastError();
     const int64_t cap = (int64_t)device_sm_count() * o;
     const int grid = (int)(p.R < cap ? p.R : cap);
-    kern<<<grid, warps * 32, 0, s>>>(p);
+    kern<<<grid, warps * 32, smem, s>>>(p);
     return cudaGetLastError();
 }
 
-template <int VPT, bool PF>
+template <int VPT, int D>
 cudaError_t launch_row_cta_vpt(const FwdParams& p, bool res, bool w32, cudaStream_t s) {
-    if (res) return w32 ? launch_row_cta<VPT, PF, true, true>(p, s)
-                        : launch_row_cta<VPT, PF, true, false>(p, s);
-    return w32 ? launch_row_cta<VPT, PF, false, true>(p, s)
-               : launch_row_cta<VPT, PF, false, false>(p, s);
+    if (res) return w32 ? launch_row_cta<VPT, D, true, true>(p, s)
+                        : launch_row_cta<VPT, D, true, false>(p, s);
+    return w32 ? launch_row_cta<VPT, D, false, true>(p, s)
+               : launch_row_cta<VPT, D, false, false>(p, s);
 }
 
 }  // namespace
+
+constexpr int kFwdRingMinRows = 32768;
 
 cudaError_t launch_fwd(const FwdParams& p, bool res, bool w32, cudaStream_t s) {
     if (p.R <= 0) return cudaSuccess;
@@ -298,8 +342,13 @@ cudaError_t launch_fwd(const FwdParams& p, bool res, bool w32, cudaStream_t s) {
     if (need <= 2) return launch_warp_vpt<2, 2>(p, res, w32, s);
     if (need <= 3) return launch_warp_vpt<3, 1>(p, res, w32, s);
     if (need <= 4) return launch_warp_vpt<4, 1>(p, res, w32, s);
-    if (p.nvec <= 512) return launch_row_cta_vpt<2, false>(p, res, w32, s);
-    return launch_row_cta_vpt<4, false>(p, res, w32, s);
+    if (p.nvec <= 512) return launch_row_cta_vpt<2, 0>(p, res, w32, s);
+    // The residual form reads two rows per row: there a two-row cp.async ring keeps enough
+    // bytes in flight to pay for itself once every CTA walks many rows (measured: H 6144 x
+    // 65537 rows 513 vs 529 us); for one input row it costs more than it brings.
+    if (res && p.R >= kFwdRingMinRows)
+        return w32 ? launch_row_cta<4, 2, true, true>(p, s) : launch_row_cta<4, 2, true, false>(p, s);
+    return launch_row_cta_vpt<4, 0>(p, res, w32, s);
 }
 
 }  // namespace rmsk

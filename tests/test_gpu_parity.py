@@ -134,6 +134,14 @@ def test_blocked_fp32_narrow_rows(H, T, residual, grid):
     run_case(T, 1, H, "bf16", seed=H + T, residual=residual, modes=(False,), grid_ctas=grid)
 
 
+@pytest.mark.parametrize("H,T,wdt,pad", [(5120, 33001, "fp32", 64), (8192, 32768, "bf16", 0)])
+def test_residual_forward_ring(H, T, wdt, pad):
+    """The residual forward of wide rows at many rows, where the rows pass through a per-thread
+    cp.async ring in shared memory: a ragged row count with FP32 weight and a padded stride,
+    and the widest row."""
+    run_case(T, 1, H, wdt, seed=H + T, residual=True, layout=(H + pad, H), modes=(False,))
+
+
 # ---- edge cases ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("H", [8, 24, 264, 776, 8192])
