@@ -271,29 +271,6 @@ def graph_time_us(fn, flush, torch, reps=20):
     return statistics.median(ts)
 
 
-def kernel_time_us(fn, flush, torch, reps=30):
-    """Kernel-active time per call: the summed device durations of this library's kernels
-    (CUPTI records through torch.profiler), L2 flushed before every call, divided by the
-    number of calls.  Used where a call lasts a few microseconds, below what CUDA events
-    around a graph replay resolve."""
-    from torch.profiler import ProfilerActivity, profile
-    fn()
-    torch.cuda.synchronize()
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        for _ in range(reps):
-            flush.zero_()
-            fn()
-        torch.cuda.synchronize()
-    total = 0.0
-    for e in prof.key_averages():
-        if "rmsk::" in e.key:
-            t = getattr(e, "device_time_total", None)
-            if t is None:
-                t = getattr(e, "cuda_time_total", 0.0)
-            total += t
-    return total / reps
-
-
 def call_spans_us(events, flush_tag="FillFunctor"):
     """Per-call spans from device records (name, start_us, end_us) of a loop that flushes L2
     before every call: records sorted by start, cut at every flush kernel; a call's span runs
