@@ -14,7 +14,8 @@
 //
 //   * rows of at most 4 vectors (16 bytes) per lane, H <= 1024: one warp per row (or per
 //     group of ROWS rows for the narrowest widths once there are rows enough to fill the
-//     GPU), a 5-level shuffle tree per row;
+//     GPU), a 5-level shuffle tree per row; for mid-sized row counts at H <= 256 the rows
+//     pass through a 4-row per-warp cp.async ring in shared memory;
 //   * wider rows: one CTA per row, every thread VPT vectors of it (2 up to H 4096, 4
 //     above), warp sums met in shared memory; in the residual form at H > 4096 and many
 //     rows, the rows pass through a two-row per-thread cp.async ring in shared memory.
@@ -140,6 +141,83 @@ __global__ void __launch_bounds__(kFwdWarpThreads) fwd_warp_kernel(const FwdPara
             if (lane == q) mine = rs[q];
         if (lane < ROWS && r0 + lane < p.R) p.rstd[r0 + lane] = mine;
     }
+}
+
+// ---- narrow rows at many rows: one warp per row, a per-warp cp.async ring ------------------------
+// Lane l owns vector l (and l + 32, ...) of every row; rows are taken grid-stride over the warps
+// of the grid.  Each warp runs an S-row ring in shared memory filled by per-lane cp.async, so S-1
+// rows of loads stay in flight per warp at no register cost; a lane reads back only what it copied
+// itself and waits for its own copies only.
+template <int VPT, int S, bool RES, bool W32>
+__global__ void __launch_bounds__(kFwdWarpThreads) fwd_warp_ring_kernel(const FwdParams p) {
+    constexpr int NTEN = RES ? 2 : 1;
+    constexpr int SB = NTEN * VPT * 512;  // one row of one warp: tensors x vectors x 32 lanes x 16 B
+    extern __shared__ __align__(16) unsigned char fsm[];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int nw = (int)(blockDim.x >> 5);
+    const float invH = 1.0f / (float)p.H;
+    unsigned char* ring = fsm + (size_t)warp * S * SB;
+    const uint32_t ring_s = smem_addr(ring);
+    const int gw = blockIdx.x * nw + warp;
+    const int nwt = gridDim.x * nw;
+    const int total = p.R > gw ? (p.R - 1 - gw) / nwt + 1 : 0;
+    auto issue = [&](int j) {
+        if (j < total) {
+            const int r = gw + j * nwt;
+            const uint32_t st = ring_s + (uint32_t)((j % S) * SB);
+            const int64_t ox = row_offset(r, p.heads, p.x.st, p.x.sk);
+            const int64_t orr = RES ? row_offset(r, p.heads, p.res.st, p.res.sk) : 0;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int v = lane + 32 * i;
+                if (v < p.nvec) {
+                    cp_async16(st + (uint32_t)(i * 512 + lane * 16), p.x.ptr + ox + 8 * v);
+                    if constexpr (RES)
+                        cp_async16(st + (uint32_t)((VPT + i) * 512 + lane * 16), p.res.ptr + orr + 8 * v);
+                }
+            }
+        }
+        cp_async_commit();  // one group per row, empty or not: wait_group counts them
+    };
+#pragma unroll
+    for (int j = 0; j < S - 1; ++j) issue(j);
+    for (int j = 0; j < total; ++j) {
+        cp_async_wait<S - 2>();  // this lane's copies of row j have landed
+        const int r = gw + j * nwt;
+        const unsigned char* st = ring + (j % S) * SB;
+        uint4 xv[VPT];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const bool in = lane + 32 * i < p.nvec;
+            xv[i] = in ? *reinterpret_cast<const uint4*>(st + i * 512 + lane * 16)
+                       : make_uint4(0u, 0u, 0u, 0u);
+        }
+        if constexpr (RES) {
+            const int64_t oh = row_offset(r, p.heads, p.h.st, p.h.sk);
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int v = lane + 32 * i;
+                if (v < p.nvec) {
+                    xv[i] = add_round8(xv[i], *reinterpret_cast<const uint4*>(st + (VPT + i) * 512 + lane * 16));
+                    st16(p.h.ptr + oh + 8 * v, xv[i]);
+                }
+            }
+        }
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) acc = __fadd_rn(acc, sumsq8(xv[i]));
+        const float rs = rsqrtf(__fmaf_rn(warp_sum(acc), invH, p.eps));
+        const int64_t oy = row_offset(r, p.heads, p.y.st, p.y.sk);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int v = lane + 32 * i;
+            if (v < p.nvec) st16(p.y.ptr + oy + 8 * v, scale8<W32>(xv[i], rs, p.w, v));
+        }
+        if (lane == 0) p.rstd[r] = rs;
+        issue(j + S - 1);
+    }
+    cp_async_wait<0>();
 }
 
 // ---- wider rows: one CTA per row ----------------------------------------------------------------
@@ -297,6 +375,25 @@ cudaError_t launch_warp_vpt(const FwdParams& p, bool res, bool w32, cudaStream_t
     return w32 ? launch_warp<VPT, 1, false, true>(p, s) : launch_warp<VPT, 1, false, false>(p, s);
 }
 
+// One warp per row with an S-row cp.async ring per warp (8-warp CTAs).
+template <int VPT, int S, bool RES, bool W32>
+cudaError_t launch_warp_ring(const FwdParams& p, cudaStream_t s) {
+    auto kern = fwd_warp_ring_kernel<VPT, S, RES, W32>;
+    const size_t smem = (size_t)(kFwdWarpThreads / 32) * S * (RES ? 2 : 1) * VPT * 512;
+    static int occ = 0;
+    if (occ == 0 && smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    const int o = resident_ctas(kern, kFwdWarpThreads, &occ, smem);
+    if (o < 0) return cudaGetLastError();
+    const int64_t need = ((int64_t)p.R + kFwdWarpThreads / 32 - 1) / (kFwdWarpThreads / 32);
+    const int64_t cap = (int64_t)device_sm_count() * o;
+    const int grid = (int)(need < cap ? need : cap);
+    kern<<<grid, kFwdWarpThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
 // One CTA per row: ceil(nvec / (32 VPT)) warps; a D-row cp.async ring when D >= 2.
 template <int VPT, int D, bool RES, bool W32>
 cudaError_t launch_row_cta(const FwdParams& p, cudaStream_t s) {
@@ -334,11 +431,20 @@ cudaError_t launch_row_cta_vpt(const FwdParams& p, bool res, bool w32, cudaStrea
 }  // namespace
 
 constexpr int kFwdRingMinRows = 32768;
+constexpr int kFwdWarpRingRows[2] = {8192, 131072};
 
 cudaError_t launch_fwd(const FwdParams& p, bool res, bool w32, cudaStream_t s) {
     if (p.R <= 0) return cudaSuccess;
     const int need = (p.nvec + 31) / 32;  // vectors per lane of a warp-wide row
-    if (need <= 1) return launch_warp_vpt<1, 4>(p, res, w32, s);
+    if (need <= 1) {
+        // Mid-sized plain forwards of rows of one vector per lane (H <= 256) keep more loads in
+        // flight through a 4-row cp.async ring per warp (measured: [1024,24,256] 7.4 vs 8.7 us,
+        // [16384,4,256] 14.4 vs 16.3 us); below the window the ring's start-up costs more than it
+        // brings, above it the register kernel's four rows per warp already saturate HBM.
+        if (!res && p.R >= kFwdWarpRingRows[0] && p.R < kFwdWarpRingRows[1])
+            return w32 ? launch_warp_ring<1, 4, false, true>(p, s) : launch_warp_ring<1, 4, false, false>(p, s);
+        return launch_warp_vpt<1, 4>(p, res, w32, s);
+    }
     if (need <= 2) return launch_warp_vpt<2, 2>(p, res, w32, s);
     if (need <= 3) return launch_warp_vpt<3, 1>(p, res, w32, s);
     if (need <= 4) return launch_warp_vpt<4, 1>(p, res, w32, s);

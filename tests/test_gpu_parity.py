@@ -142,6 +142,15 @@ def test_residual_forward_ring(H, T, wdt, pad):
     run_case(T, 1, H, wdt, seed=H + T, residual=True, layout=(H + pad, H), modes=(False,))
 
 
+@pytest.mark.parametrize("H,T,pad", [(24, 8192, 8), (256, 131071, 0), (136, 20000, 64)])
+def test_narrow_forward_ring(H, T, pad):
+    """Rows of one vector per lane at mid-sized row counts, where the forward passes rows
+    through a per-warp cp.async ring: a 24-wide row (most lanes idle), the window's first
+    row count and a padded stride, and a ragged count just below the window's end."""
+    run_case(T, 1, H, "fp32" if H % 48 == 0 else "bf16", seed=H + T, layout=(H + pad, H),
+             modes=(False,))
+
+
 # ---- edge cases ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("H", [8, 24, 264, 776, 8192])
