@@ -70,7 +70,7 @@ def run_case(T, heads, H, wdt, seed=0, family="F1", residual=False, modes=(True,
     return out, dw_ref
 
 
-# ---- BASELINE configurations -----------------------------------------------------------
+# ---- the configurations of the pages' tables -------------------------------------------
 
 def test_tiny_config():
     """T=64, H=512, x BF16 N(0,1), FP32 weight 1+0.1N(0,1), dy N(0,1), eps 1e-6; fwd then
