@@ -29,7 +29,8 @@ def _call_noalloc(L, x, w, rstd, dy, dx, dw):
     _lib.check(rc)
 
 
-@pytest.mark.parametrize("T,H,wdt", [(4099, 6144, "bf16"), (20000, 1536, "fp32")])
+@pytest.mark.parametrize("T,H,wdt", [(4099, 6144, "bf16"), (20000, 1536, "fp32"),
+                                      (30000, 256, "bf16")])
 def test_noalloc_backward_matches_the_workspace_backward(T, H, wdt):
     L = _lib.lib()
     x = dev_rows(synth.rows(21, "x", T, H))
