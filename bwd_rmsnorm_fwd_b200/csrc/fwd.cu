@@ -4,10 +4,9 @@
 //   residual form: h_rj = BF16(x_rj + res_rj), h is stored and the norm runs on h.
 // (flashinfer PR #8848 introduction and "Workload"; PR #8512 "Residual rows".)
 //
-// Design: every row is read from HBM once into registers, reduced, scaled and written
-// back.  The forward reads a row once and writes it
-// once, so what sets its speed is how many bytes are in flight per SM and how little
-// work sits between a row's last load and its first store.  Many small resident CTAs with
+// Design: every row is read from HBM once, reduced, scaled and written back once, so what
+// sets the forward's speed is how many bytes are in flight per SM and how little work sits
+// between a row's last load and its first store.  Many small resident CTAs with
 // all of a row's loads issued before any use beat a shared-memory pipeline with one CTA
 // per SM at every width and row count measured (H 256..8192, rows 1..393216), because the
 // pipeline's per-row reduction, barrier and wait latencies stay exposed with few warps.
@@ -25,7 +24,8 @@
 // each 16-byte vector is summed as a small tree, a thread sums its vectors in order, then a
 // shuffle tree (and, across warps, a sum in warp order).  rstd = rsqrtf(sum * (1/H) + eps)
 // in FP32: CUDA documents rsqrtf to within 2 ulp and the FMA rounds the mean once, so rstd
-// is within a few FP32 ulps of the exact value.  The forward has no device-side waits.
+// is within a few FP32 ulps of the exact value.  The forward has no barrier waits: the rings
+// wait only for a thread's own copies to land.
 #include "common.cuh"
 
 namespace rmsk {
