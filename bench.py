@@ -8,14 +8,18 @@ and seeded.  Inputs are far larger than L2 and L2 is also flushed before every t
 step.  ``value`` is microseconds per step (lower is better); the pages report 1640.48 us
 for this step on B200 (flashinfer PR #8848 table, H6144 T131072, BF16 weight).
 
-Every launch inside the timed region is one of librmsnorm_train's kernels.  The JSON
-line also carries the roofline of the dominant kernel (the backward), the CPU oracle
-as a baseline, an end-to-end figure with host buffers, SM clocks sampled during the
-timed region, and a per-configuration table (CUPTI span of a CUDA-graph replay, cold L2,
-the pages' timing rule) with the achieved fraction of the measured HBM bandwidth.
+Every launch inside the timed region is one of librmsnorm_train's kernels.  Output: one
+JSON line on stdout, printed last and kept short (under MAX_LINE_BYTES): the step time, the
+roofline of the dominant kernel (the backward), the CPU oracle as a baseline (all host
+threads and one thread), an end-to-end figure with host buffers, SM clocks sampled during
+the timed region, and a summary of the per-configuration table.  The table itself (every
+configuration of the pages' tables: median, p10 and p90 of the CUPTI span of a CUDA-graph
+replay with L2 flushed before each, 3 interleaved rounds x 67 replays per call, an A/A
+floor per group, and the fraction of the measured HBM bandwidth) goes to its own file,
+``--per-config-out``.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-       [--sweep all|none]
+       [--sweep all|none|<group>] [--per-config-out FILE]
 For N > 1 launch under torchrun: every rank runs its own replica (weak scaling, no
 collective on the data path); the step time is the maximum over ranks.
 """
@@ -159,13 +163,16 @@ class ClockSampler:
 
 # ---- the reference arm: the FP64 CPU oracle ----------------------------------------------------
 
-def oracle_step_seconds(rows, H, nthreads=0):
-    """One checkpointed step (fwd, fwd, bwd) of the oracle on `rows` rows of width H."""
-    import oracle
+def oracle_inputs(rows, H):
     from bwd_rmsnorm_fwd_b200 import synth
-    x = synth.rows(0, "x", rows, H)
-    dy = synth.rows(0, "dy", rows, H)
-    w = synth.weight(0, H, "bf16")
+    return synth.rows(0, "x", rows, H), synth.rows(0, "dy", rows, H), synth.weight(0, H, "bf16")
+
+
+def oracle_step_seconds(inputs, nthreads=0):
+    """One checkpointed step (fwd, fwd, bwd) of the oracle on the given rows; nthreads = 0
+    uses every hardware thread."""
+    import oracle
+    x, dy, w = inputs
     t0 = time.perf_counter()
     oracle.train_fwd(x, w, 1e-6, nthreads=nthreads)
     _, rstd = oracle.train_fwd(x, w, 1e-6, nthreads=nthreads)
@@ -173,21 +180,32 @@ def oracle_step_seconds(rows, H, nthreads=0):
     return time.perf_counter() - t0
 
 
-def oracle_sample_rows(target_s):
-    t = oracle_step_seconds(256, HEAD_H)
-    rows = int(256 * target_s / max(t, 1e-6))
-    return max(256, min(HEAD_T, rows))
+def oracle_sample_rows(target_s, nthreads=0):
+    """Rows of the headline width that one oracle step covers in about target_s seconds."""
+    probe = 256 if nthreads != 1 else 64
+    t = oracle_step_seconds(oracle_inputs(probe, HEAD_H), nthreads)
+    rows = int(probe * target_s / max(t, 1e-6))
+    return max(probe, min(HEAD_T, rows))
 
 
 def cpu_baseline(target_s=10.0):
+    """The oracle, as it stands, on a bounded row sample of the headline step, with every
+    hardware thread and with one thread; each scaled linearly to all rows."""
     import oracle
-    rows = oracle_sample_rows(target_s)
-    t = oracle_step_seconds(rows, HEAD_H)
-    us = t * (HEAD_T / rows) * 1e6
-    return {"value": round(us, 1), "unit": "us", "cores": oracle.hardware_threads(),
-            "kind": "oracle",
-            "sample": f"{rows} of {HEAD_T} rows of the headline step (fwd, fwd, bwd) on the "
-                      f"FP64 C++ oracle, {t:.1f} s, scaled linearly to all rows"}
+    out = None
+    for nthreads in (0, 1):
+        rows = oracle_sample_rows(target_s, nthreads)
+        t = oracle_step_seconds(oracle_inputs(rows, HEAD_H), nthreads)
+        cores = oracle.hardware_threads() if nthreads == 0 else 1
+        rec = {"value": round(t * (HEAD_T / rows) * 1e6, 1), "unit": "us", "cores": cores,
+               "kind": "oracle",
+               "sample": f"{rows} of {HEAD_T} rows of the headline step (fwd, fwd, bwd), "
+                         f"{t:.1f} s, scaled linearly to all rows"}
+        if out is None:
+            out = rec
+        else:
+            out["single_thread"] = {k: rec[k] for k in ("value", "cores", "sample")}
+    return out
 
 
 def run_reference(args):
@@ -196,18 +214,21 @@ def run_reference(args):
         return 0
     import oracle
     oracle.build()
-    # per-step sample sized so that warmup + steps take about two minutes in all
+    # per-step sample sized so that warmup + steps take about two minutes in all; the
+    # inputs are drawn once and every step recomputes from them
     rows = oracle_sample_rows(min(3.0, 120.0 / (args.steps + args.warmup)))
+    inputs = oracle_inputs(rows, HEAD_H)
     for _ in range(args.warmup):
-        oracle_step_seconds(rows, HEAD_H)
-    ts = [oracle_step_seconds(rows, HEAD_H) for _ in range(args.steps)]
+        oracle_step_seconds(inputs)
+    ts = [oracle_step_seconds(inputs) for _ in range(args.steps)]
     us = statistics.median(ts) * (HEAD_T / rows) * 1e6
     line = {
         "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": "us",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(us / 1e3, 3), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "l2": "inputs larger than L2"},
+        "config": {"workload": WORKLOAD, "T": HEAD_T, "H": HEAD_H, "w": "bf16",
+                   "l2": "inputs larger than L2"},
         "cpu_baseline": {"value": round(us, 1), "unit": "us", "cores": oracle.hardware_threads(),
                          "kind": "oracle",
                          "sample": f"{rows} of {HEAD_T} rows per step, scaled linearly"},
@@ -244,33 +265,6 @@ def make_inputs(T, H, wdt, seed, device, torch):
     return x, dy, w
 
 
-def graph_time_us(fn, flush, torch, reps=20):
-    """Median per-replay time of fn captured in a CUDA graph, L2 flushed before every
-    replay (outside the timed events)."""
-    fn()  # warm: allocates outputs / workspace outside the capture
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    try:
-        with torch.cuda.graph(g):
-            fn()
-        run = g.replay
-    except Exception:
-        run = fn
-    ts = []
-    for i in range(reps + 3):
-        flush.zero_()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record()
-        run()
-        b.record()
-        b.synchronize()
-        if i >= 3:
-            ts.append(a.elapsed_time(b) * 1e3)
-    del g
-    return statistics.median(ts)
-
-
 def call_spans_us(events, flush_tag="FillFunctor"):
     """Per-call spans from device records (name, start_us, end_us) of a loop that flushes L2
     before every call: records sorted by start, cut at every flush kernel; a call's span runs
@@ -289,58 +283,125 @@ def call_spans_us(events, flush_tag="FillFunctor"):
     return spans
 
 
-def span_time_us(fn, flush, torch, reps=30):
-    """Median CUPTI span of one call replayed from a CUDA graph with L2 flushed before each
-    replay (the pages' timing rule): first kernel start to last kernel end, every kernel of
-    the call inside the span."""
+def interleaved_order(keys, rounds, reps):
+    """Replay order of the timing protocol: `rounds` rounds; in round r the calls run in the
+    list's order rotated by r; each call `reps` times in a row."""
+    order = []
+    n = len(keys)
+    for r in range(rounds):
+        k = r % n if n else 0
+        for key in keys[k:] + keys[:k]:
+            order.extend([key] * reps)
+    return order
+
+
+def quantile(xs, q):
+    s = sorted(xs)
+    if not s:
+        return None
+    i = q * (len(s) - 1)
+    lo = int(i)
+    hi = min(lo + 1, len(s) - 1)
+    return s[lo] + (s[hi] - s[lo]) * (i - lo)
+
+
+def time_group(calls, flush, torch, rounds=3, reps=67):
+    """CUPTI spans of several calls, each captured in its own CUDA graph and replayed with L2
+    flushed before every replay, in interleaved rounds (the pages' protocol: rounds x reps
+    replays per call, rotated order).  `calls` is a list of (key, fn); every call runs once
+    before any capture, so a growing workspace reaches its size outside the captures.
+    Returns {key: [span_us, ...]}."""
     from torch.autograd import DeviceType
     from torch.profiler import ProfilerActivity, profile
-    fn()
+    for _, fn in calls:
+        fn()
     torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    try:
+    graphs = {}
+    for key, fn in calls:
+        g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             fn()
-        run = g.replay
-    except Exception:
-        run = fn
-    run()
+        graphs[key] = g
+    for g in graphs.values():
+        g.replay()
     torch.cuda.synchronize()
+    order = interleaved_order([k for k, _ in calls], rounds, reps)
     with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        for _ in range(reps):
+        for key in order:
             flush.zero_()
-            run()
+            graphs[key].replay()
         torch.cuda.synchronize()
     events = [(e.name, e.time_range.start, e.time_range.end) for e in prof.events()
               if e.device_type == DeviceType.CUDA]
-    del g
     spans = call_spans_us(events)
-    if not spans:
-        raise RuntimeError("the profiler recorded no device activity for the call")
-    return statistics.median(spans)
+    del graphs
+    if len(spans) != len(order):
+        raise RuntimeError(f"profiler gave {len(spans)} call spans for {len(order)} replays")
+    out = {k: [] for k, _ in calls}
+    for key, s in zip(order, spans):
+        out[key].append(s)
+    return out
 
 
-SWEEP_GROUPS = ("tiny", "small-T", "residual", "per-head", "large-T")
+def event_time_us(fn, flush, torch, reps=20):
+    """Median CUDA-event time of fn's graph replay on the current stream, L2 flushed before
+    every replay (outside the events)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    ts = []
+    for i in range(reps + 3):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        b.synchronize()
+        if i >= 3:
+            ts.append(a.elapsed_time(b) * 1e3)
+    del g
+    return statistics.median(ts)
 
 
-def sweep(torch, api, flush, peak, dev, groups=SWEEP_GROUPS):
-    """Per-configuration table: us per call (CUPTI span of a graph replay, cold L2; CUDA events
-    around the replay too where a call is long enough) and the fraction of the measured HBM
-    bandwidth, for every configuration of the pages' tables."""
+SWEEP_GROUPS = ("tiny", "small-T", "residual", "per-head", "large-T", "long-256")
+
+
+def sweep(torch, api, flush, peak, dev, groups=SWEEP_GROUPS, rounds=3, reps=67):
+    """Per-configuration table for every configuration of the pages' tables: us per call
+    (median, p10 and p90 of the CUPTI span of a CUDA-graph replay, cold L2, rounds x reps
+    replays in interleaved rounds), an A/A floor per group (the group's first call captured
+    twice and timed as two programs), CUDA-event time of the replay where a call is long
+    enough, and the fraction of the measured HBM bandwidth."""
     out = []
     ws = api.Workspace(dev)
 
-    def rec(cfg, form, H, T, wdt, op, fn, nbytes, replay):
-        us = span_time_us(fn, flush, torch)
-        gbs = nbytes / (us * 1e-6) / 1e9
-        row = {"cfg": cfg, "form": form, "H": H, "T": T, "w": wdt, "op": op,
-               "us": round(us, 2), "gbs": round(gbs, 1), "frac": round(gbs / peak, 3),
-               "timer": "cupti_span"}
-        if replay:
-            row["replay_us"] = round(graph_time_us(fn, flush, torch), 2)
-        out.append(row)
+    def run_group(entries):
+        # entries: (meta, fn, nbytes, replay); the first call is also timed as its own A/A twin
+        calls = [(i, e[1]) for i, e in enumerate(entries)]
+        calls.append(("aa", entries[0][1]))
+        spans = time_group(calls, flush, torch, rounds, reps)
+        m0, ma = statistics.median(spans[0]), statistics.median(spans["aa"])
+        aa = abs(m0 - ma) / ((m0 + ma) / 2)
+        for i, (meta, fn, nbytes, replay) in enumerate(entries):
+            us = statistics.median(spans[i])
+            gbs = nbytes / (us * 1e-6) / 1e9
+            row = dict(meta)
+            row.update({"us": round(us, 2), "p10": round(quantile(spans[i], 0.1), 2),
+                        "p90": round(quantile(spans[i], 0.9), 2), "gbs": round(gbs, 1),
+                        "frac": round(gbs / peak, 3), "timer": "cupti_span",
+                        "replays": len(spans[i])})
+            if i == 0:
+                row["aa_floor"] = round(aa, 4)
+            if replay:
+                row["replay_us"] = round(event_time_us(fn, flush, torch), 2)
+            out.append(row)
+        torch.cuda.synchronize()
 
-    def ops(cfg, form, x, dy, w, H, T, R, wdt, heads=1, res=None, dh=None, do=("fwd", "det", "nondet")):
+    def ops(entries, cfg, form, x, dy, w, H, T, R, wdt, res=None, dh=None,
+            do=("fwd", "det", "nondet")):
         wb = 2 if wdt == "bf16" else 4
         isres = res is not None
         # CUDA events around a graph replay as well, where a call outlasts the launch latency
@@ -350,36 +411,42 @@ def sweep(torch, api, flush, peak, dev, groups=SWEEP_GROUPS):
         else:
             _, rstd = api.rmsnorm_train_fwd(x, w)
             h = x
+        meta = {"cfg": cfg, "form": form, "H": H, "T": T, "w": wdt}
         if "fwd" in do:
-            rec(cfg, form, H, T, wdt, "fwd", lambda: api.rmsnorm_train_fwd(x, w, residual=res),
-                bytes_fwd(R, H, wb, isres), replay)
+            entries.append((dict(meta, op="fwd"),
+                            lambda: api.rmsnorm_train_fwd(x, w, residual=res),
+                            bytes_fwd(R, H, wb, isres), replay))
         for det in (True, False):
             if ("det" if det else "nondet") not in do:
                 continue
-            rec(cfg, form, H, T, wdt, "bwd_det" if det else "bwd_nondet",
-                lambda: api.rmsnorm_train_bwd(h, w, rstd, dy, deterministic=det, dh=dh,
-                                              workspace=ws),
-                bytes_bwd(R, H, wb, isres), replay)
+            entries.append((dict(meta, op="bwd_det" if det else "bwd_nondet"),
+                            (lambda d: lambda: api.rmsnorm_train_bwd(
+                                h, w, rstd, dy, deterministic=d, dh=dh, workspace=ws))(det),
+                            bytes_bwd(R, H, wb, isres), replay))
 
-    # Tiny and small-T sweep (deterministic backward, single launch)
     if "tiny" in groups:
+        e = []
         x, dy, w = make_inputs(64, 512, "fp32", 1, dev, torch)
-        ops("tiny", "plain", x, dy, w, 512, 64, 64, "fp32", do=("fwd", "det"))
+        ops(e, "tiny", "plain", x, dy, w, 512, 64, 64, "fp32", do=("fwd", "det"))
+        run_group(e)
     for H in (256, 512, 2048, 4096) if "small-T" in groups else ():
         for wdt in ("bf16", "fp32"):
+            e = []
             xa, dya, w = make_inputs(227, H, wdt, 2, dev, torch)
             for T in (1, 2, 8, 32, 87, 227):
-                ops("small-T", "plain", xa[:T], dya[:T], w, H, T, T, wdt, do=("det",))
-    # residual H 6144
+                ops(e, "small-T", "plain", xa[:T], dya[:T], w, H, T, T, wdt, do=("det",))
+            run_group(e)
     for T in (32, 4096, 65537) if "residual" in groups else ():
+        e = []
         x, dy, w = make_inputs(T, 6144, "bf16", 3, dev, torch)
         res, dh, _ = make_inputs(T, 6144, "bf16", 4, dev, torch)
-        ops("residual", "res", x, dy, w, 6144, T, T, "bf16", res=res, dh=dh)
-        del x, dy, res, dh
-    # per-head views, FP32 weight
+        ops(e, "residual", "res", x, dy, w, 6144, T, T, "bf16", res=res, dh=dh)
+        run_group(e)
+        del e, x, dy, res, dh
     for T in (1024, 16384) if "per-head" in groups else ():
         for name, heads, st, sk in (("24x256_pages", 24, 12288, 512),
                                     ("24x256_dense", 24, 6144, 256), ("4x256", 4, 1024, 256)):
+            e = []
             n = (T - 1) * st + (heads - 1) * sk + 256
             g = torch.Generator(device=dev)
             g.manual_seed(5)
@@ -388,16 +455,109 @@ def sweep(torch, api, flush, peak, dev, groups=SWEEP_GROUPS):
             x = torch.as_strided(bx, (T, heads, 256), (st, sk, 1))
             dy = torch.as_strided(bd, (T, heads, 256), (st, sk, 1))
             w = 1 + 0.1 * torch.randn(256, generator=g, device=dev)
-            ops("per-head", name, x, dy, w, 256, T, T * heads, "fp32", heads=heads)
-            del bx, bd
-    # large T
+            ops(e, "per-head", name, x, dy, w, 256, T, T * heads, "fp32")
+            run_group(e)
+            del e, bx, bd
     for H in (1536, 2048, 4096, 5120, 6144) if "large-T" in groups else ():
         for wdt in ("bf16", "fp32"):
+            e = []
             xa, dya, w = make_inputs(131072, H, wdt, 6, dev, torch)
             for T in (65537, 98304, 131072):
-                ops("large-T", "plain", xa[:T], dya[:T], w, H, T, T, wdt)
-            del xa, dya
+                ops(e, "large-T", "plain", xa[:T], dya[:T], w, H, T, T, wdt)
+            run_group(e)
+            del e, xa, dya
+            torch.cuda.empty_cache()
+    if "long-256" in groups:
+        # the very long narrow-row regime: H 256 rows at T 1048576, both weight dtypes
+        for wdt in ("bf16", "fp32"):
+            e = []
+            x, dy, w = make_inputs(1048576, 256, wdt, 7, dev, torch)
+            ops(e, "long-256", "plain", x, dy, w, 256, 1048576, 1048576, wdt)
+            run_group(e)
+            del e, x, dy
+    torch.cuda.empty_cache()
     return out
+
+
+def per_config_summary(rows):
+    """Worst fraction of the measured bandwidth per large-T operation, and the largest A/A
+    floor: the few figures of the table that go into the headline line."""
+    s = {}
+    for op in ("fwd", "bwd_det", "bwd_nondet"):
+        fr = [r["frac"] for r in rows if r["cfg"] == "large-T" and r["op"] == op]
+        if fr:
+            s[f"large_T_min_frac_{op}"] = min(fr)
+    aa = [r["aa_floor"] for r in rows if "aa_floor" in r]
+    if aa:
+        s["aa_floor_max"] = max(aa)
+    return s
+
+
+MAX_LINE_BYTES = 3000
+
+
+def emit(line, per_cfg=None, per_cfg_path=None, peak=None, peak_kind=None, clocks=None,
+         stream=None):
+    """Writes the per-configuration table (when there is one) to its own file and prints the
+    headline JSON line last, on its own, on stdout.  The table stays out of the line, which
+    must fit in MAX_LINE_BYTES."""
+    stream = stream or sys.stdout
+    if per_cfg is not None:
+        line["per_config"] = dict(per_config_summary(per_cfg), rows=len(per_cfg),
+                                  file=os.path.relpath(per_cfg_path, ROOT) if per_cfg_path else None)
+        if per_cfg_path:
+            os.makedirs(os.path.dirname(os.path.abspath(per_cfg_path)), exist_ok=True)
+            with open(per_cfg_path, "w") as f:
+                json.dump({"peak_gbs": peak, "peak_kind": peak_kind, "clocks": clocks,
+                           "timer": "CUPTI span of a CUDA-graph replay, L2 flushed before each "
+                                    "replay; 3 interleaved rounds x 67 replays per call",
+                           "rows": per_cfg}, f, indent=0)
+    text = json.dumps(line, separators=(",", ":"))
+    if len(text) > MAX_LINE_BYTES:
+        raise RuntimeError(f"headline line of {len(text)} bytes exceeds {MAX_LINE_BYTES}")
+    stream.write(text + "\n")
+    stream.flush()
+    return text
+
+
+def headline_line(m):
+    """The headline JSON object from the measured quantities `m` (R, H, det, world, steps,
+    warmup, us_step, bwd_us, e2e_us, peak, peak_kind, clocks, cpu)."""
+    R, H, wb, det = m["R"], m["H"], 2, m["det"]
+    head = (R, H) == (HEAD_T, HEAD_H)
+    us_step = m["us_step"]
+    step_bytes = 2 * bytes_fwd(R, H, wb) + bytes_bwd(R, H, wb)
+    bwd_bytes = bytes_bwd(R, H, wb)
+    achieved = bwd_bytes / (m["bwd_us"] * 1e-6) / 1e9
+    clocks = m["clocks"] or {}
+    return {
+        "metric": METRIC, "value": round(us_step, 2), "unit": "us", "n_gpus": m["world"],
+        "steps": m["steps"], "warmup": m["warmup"], "ms_per_step": round(us_step / 1e3, 4),
+        "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": (round(us_step / (PAGES_STEP_DET_US if det else PAGES_STEP_US), 4)
+                        if head else None),
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD if head else
+                   f"checkpointed step at T={R}, H={H} (reduced case)",
+                   "T": R, "H": H, "w": "bf16", "deterministic": det,
+                   "parallelism": f"replicas x{m['world']}" if m["world"] > 1 else "single GPU",
+                   "l2": "inputs larger than L2, and L2 flushed before every step"},
+        "step_gbs": round(step_bytes / (us_step * 1e-6) / 1e9, 1),
+        "aggregate_gbs": round(m["world"] * step_bytes / (us_step * 1e-6) / 1e9, 1),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": m["peak"],
+                     "unit": "GB/s", "frac": round(achieved / m["peak"], 4),
+                     "peak_kind": m["peak_kind"],
+                     "kernel": f"backward (deterministic={det}), H{H} T{R}",
+                     "bytes_per_launch": bwd_bytes, "launch_us": round(m["bwd_us"], 2),
+                     "traffic": recorded_traffic(
+                         f"bwd_{'det' if det else 'nondet'}_h{H}_t{R}_bf16")},
+        "e2e": {"value": round(m["e2e_us"], 1) if m["e2e_us"] else None, "unit": "us",
+                "h2d_bytes_per_step": 2 * R * H * 2,
+                "d2h_bytes_per_step": R * H * 2 + H * 4},
+        "gpu_launches": (4 if det else 3) * m["steps"],
+        "clocks": {k: clocks.get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons", "power_w_max")},
+        "cpu_baseline": m["cpu"],
+    }
 
 
 def main():
@@ -408,6 +568,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sweep", default="all", choices=["all", "none", *SWEEP_GROUPS],
                     help="per-configuration table: every group, none, or one group")
+    ap.add_argument("--per-config-out", default=os.path.join(ROOT, "profiles",
+                                                             "per_config_b200.json"),
+                    help="file the per-configuration table is written to")
     ap.add_argument("--det", action="store_true",
                     help="the step's backward uses deterministic=True")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -438,7 +601,7 @@ def main():
     peak, peak_kind = peaks()
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > L2
 
-    R, H, wb = args.rows, args.width, 2
+    R, H = args.rows, args.width
     x, dy, w = make_inputs(R, H, "bf16", 1234 + rank, dev, torch)
     ws = api.Workspace(dev)
 
@@ -477,9 +640,6 @@ def main():
     ms_step = max_over_ranks(sum(step_us) / len(step_us) / 1e3, dist, dev)
     us_step = ms_step * 1e3
     bwd_avg_us = sum(bwd_us) / len(bwd_us)
-    step_bytes = 2 * bytes_fwd(R, H, wb) + bytes_bwd(R, H, wb)
-    bwd_bytes = bytes_bwd(R, H, wb)
-    achieved = bwd_bytes / (bwd_avg_us * 1e-6) / 1e9
 
     # end to end through the public API with pinned host buffers
     xh = x.cpu().pin_memory()
@@ -508,7 +668,9 @@ def main():
     e2e_us = statistics.median(e2e) if e2e else None
 
     per_cfg = None
-    if args.sweep != "none" and rank == 0:
+    # the per-configuration table is a single-GPU measurement: with several ranks the others
+    # would wait for it in the closing barrier
+    if args.sweep != "none" and world == 1:
         del x, dy
         torch.cuda.empty_cache()
         per_cfg = sweep(torch, api, flush, peak, dev,
@@ -519,38 +681,12 @@ def main():
         cpu = cpu_baseline(10.0)
 
     if rank == 0:
-        line = {
-            "metric": METRIC, "value": round(us_step, 2), "unit": "us", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-            "higher_is_better": False, "scaling": "weak",
-            "vs_baseline": (round(us_step / (PAGES_STEP_DET_US if args.det else PAGES_STEP_US), 4)
-                            if (R, H) == (HEAD_T, HEAD_H) else None),
-            "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": (WORKLOAD if (R, H) == (HEAD_T, HEAD_H) else
-                                    f"checkpointed step at T={R}, H={H} (reduced case)")
-                       + f", backward deterministic={args.det}", "T": R, "H": H,
-                       "w": "bf16",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2, and L2 flushed before every step"},
-            "step_gbs": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
-            "aggregate_gbs": round(world * step_bytes / (ms_step * 1e-3) / 1e9, 1),
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                         "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "peak_kind": peak_kind,
-                         "kernel": f"bwd_staged_kernel (deterministic={args.det}), H{H} T{R}",
-                         "bytes_per_launch": bwd_bytes, "launch_us": round(bwd_avg_us, 2),
-                         "traffic": recorded_traffic(
-                             f"bwd_{'det' if args.det else 'nondet'}_h{H}_t{R}_bf16")},
-            "e2e": {"value": round(e2e_us, 1) if e2e_us else None, "unit": "us",
-                    "h2d_bytes_per_step": 2 * R * H * 2,
-                    "d2h_bytes_per_step": R * H * 2 + H * 4},
-            "gpu_launches": (4 if args.det else 3) * args.steps,
-            "clocks": clocks,
-            "cpu_baseline": cpu,
-        }
-        if per_cfg is not None:
-            line["per_config"] = per_cfg
-        print(json.dumps(line))
+        line = headline_line(dict(
+            R=R, H=H, det=bool(args.det), world=world, steps=args.steps, warmup=args.warmup,
+            us_step=us_step, bwd_us=bwd_avg_us, e2e_us=e2e_us, peak=peak, peak_kind=peak_kind,
+            clocks=clocks, cpu=cpu))
+        emit(line, per_cfg, args.per_config_out if per_cfg is not None else None, peak,
+             peak_kind, clocks)
     if dist:
         dist.barrier()
         dist.destroy_process_group()

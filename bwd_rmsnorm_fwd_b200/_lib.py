@@ -51,6 +51,7 @@ SIGNATURES = [
       _vp]),
     ("rms_train_bwd_noalloc", _i32,
      [RmsShape, RmsRows, _vp, _i32, _vp, RmsRows, RmsRows, _vp, _vp]),
+    ("rms_noalloc_status", _i32, [_vp]),
     ("rms_train_bwd_workspace_bytes", _sz, [RmsShape, _i32, _i32]),
     ("rms_det_plan", _i32, [RmsShape, ctypes.POINTER(ctypes.c_int32),
                             ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),

@@ -19,7 +19,8 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "librmsnorm_train.so")
 
 SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "noalloc.cu", "tma.cu"]
-HEADERS = [os.path.join(CSRC, "common.cuh"), os.path.join(INCLUDE, "rmsnorm_train.h")]
+HEADERS = [os.path.join(CSRC, "common.cuh"), os.path.join(CSRC, "launch_cache.h"),
+           os.path.join(INCLUDE, "rmsnorm_train.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

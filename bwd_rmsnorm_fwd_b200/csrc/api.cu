@@ -1,5 +1,6 @@
 // C ABI of librmsnorm_train: argument checks, workspace layout, program choice.
 // The declarations and their contract are in include/rmsnorm_train.h.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -40,8 +41,9 @@ constexpr size_t kWsHeader = 256;  // status word, ticket
 // it, never land on it whatever the H of the call that wrote them.
 constexpr size_t kAccBytes = (size_t)kMaxH * 8;
 
-int64_t g_small_rows_override = -1;
-int64_t g_wait_cycles = rmsk::kDefaultWaitCycles;
+// process-wide settings (rms_set_small_rows_limit, rms_set_wait_limit_cycles)
+std::atomic<int64_t> g_small_rows_override{-1};
+std::atomic<int64_t> g_wait_cycles{rmsk::kDefaultWaitCycles};
 
 struct Span {
     uintptr_t lo, hi;  // [lo, hi)
@@ -138,7 +140,8 @@ int64_t default_small_rows(int H) {
 }
 
 bool use_small(int64_t R, int H) {
-    const int64_t lim = g_small_rows_override >= 0 ? g_small_rows_override : default_small_rows(H);
+    const int64_t ov = g_small_rows_override.load();
+    const int64_t lim = ov >= 0 ? ov : default_small_rows(H);
     return R <= lim && R <= 2048;
 }
 
@@ -167,7 +170,8 @@ size_t ws_bytes(const rms_shape& s, int det) {
 
 int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const float* rstd,
                rms_rows dy, const rms_rows* dh, rms_rows dx, float* dw, int deterministic,
-               void* ws, size_t ws_size, int grid_ctas, void* stream) {
+               void* ws, size_t ws_size, int grid_ctas, void* stream,
+               rmsk::PreLaunchFn hook = nullptr, void* hook_ctx = nullptr) {
     int rc = check_shape(shape);
     if (rc) return rc;
     if (w_dtype != RMS_BF16 && w_dtype != RMS_FP32)
@@ -236,9 +240,10 @@ int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const fl
     p.blocks_per_chunk = plan.L;
     p.fold_segments = plan.S;
     p.n_chunks = plan.n_chunks;
-    p.wait_cycles = g_wait_cycles;
+    p.wait_cycles = g_wait_cycles.load();
     const bool res = dh != nullptr;
     const bool w32 = w_dtype == RMS_FP32;
+    if (hook && (rc = hook(hook_ctx, st))) return rc;
     cudaError_t e;
     if (use_small(R, H)) {
         e = rmsk::launch_bwd_small(p, res, w32, st);
@@ -260,17 +265,29 @@ int set_error(int code, const char* msg) {
     return code;
 }
 
-int device_sm_count() {
-    static int cached[64];
+int bwd_entry(rms_shape shape, rms_rows x, const void* w, int w_dtype, const float* rstd,
+              rms_rows dy, const rms_rows* dh, rms_rows dx, float* dw, int deterministic,
+              void* ws, size_t ws_bytes, int grid_ctas, void* stream, PreLaunchFn hook,
+              void* hook_ctx) {
+    return bwd_common(shape, x, w, w_dtype, rstd, dy, dh, dx, dw, deterministic, ws, ws_bytes,
+                      grid_ctas, stream, hook, hook_ctx);
+}
+
+int current_device() {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!cached[dev]) {
+    return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
+int device_sm_count() {
+    static PerDevice<1> cached;
+    const int dev = current_device();
+    if (dev < 0) return 148;
+    return cached.get(dev, 0, [dev]() {
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
             n = 148;
-        cached[dev] = n;
-    }
-    return cached[dev];
+        return n;
+    });
 }
 
 }  // namespace rmsk
@@ -385,15 +402,11 @@ int rms_train_bwd_path(rms_shape shape, int deterministic) {
 }
 
 int64_t rms_set_small_rows_limit(int64_t rows) {
-    const int64_t prev = g_small_rows_override;
-    g_small_rows_override = rows < 0 ? -1 : rows;
-    return prev;
+    return g_small_rows_override.exchange(rows < 0 ? -1 : rows);
 }
 
 int64_t rms_set_wait_limit_cycles(int64_t cycles) {
-    const int64_t prev = g_wait_cycles;
-    g_wait_cycles = cycles < 0 ? rmsk::kDefaultWaitCycles : cycles;
-    return prev;
+    return g_wait_cycles.exchange(cycles < 0 ? rmsk::kDefaultWaitCycles : cycles);
 }
 
 int rms_status(void* workspace, void* stream) {

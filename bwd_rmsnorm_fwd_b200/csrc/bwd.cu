@@ -928,13 +928,9 @@ cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
         return cudaErrorInvalidConfiguration;  // the slot totals must fit in the ring
     sc.n_stages = ns;
     const size_t smem = (size_t)sc.stage_offset + (size_t)ns * sc.stage_bytes;
-    static size_t smem_set = 0;
-    if (smem > smem_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        smem_set = smem;
-    }
+    static SmemGrant granted;
+    cudaError_t ge = grant_smem(granted, current_device(), kern, smem);
+    if (ge != cudaSuccess) return ge;
     int grid = grid_ctas;
     if (grid <= 0) {
         const int64_t cap = device_sm_count();
@@ -961,16 +957,14 @@ cudaError_t launch_warp_bwd(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     const size_t ring = (size_t)nw * S * warp_stage_bytes<VPT, RES>();
     const size_t smem = (size_t)nw * p.H * sizeof(double) + ring;
     const size_t smem_max = (size_t)nw * 256 * VPT * sizeof(double) + ring;  // widest row
-    static int occ = 0;  // resident CTAs per SM at the widest row of this instantiation
-    if (occ == 0) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem_max);
-        if (e != cudaSuccess) return e;
-        int o = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, nw * 32, smem_max);
-        if (e != cudaSuccess) return e;
-        occ = o > 0 ? o : 1;
-    }
+    // resident CTAs per SM at the widest row of this instantiation, per device
+    static SmemGrant granted;
+    static PerDevice<1> occ_cache;
+    const int dev = current_device();
+    cudaError_t e = grant_smem(granted, dev, kern, smem_max);
+    if (e != cudaSuccess) return e;
+    const int occ = resident_ctas(occ_cache, dev, 0, kern, nw * 32, smem_max, &e);
+    if (occ < 0) return e;
     int grid = grid_ctas;
     if (grid <= 0) {
         int64_t need = ((int64_t)p.R + nw - 1) / nw;
@@ -1051,12 +1045,10 @@ cudaError_t launch_small_t(const BwdParams& p, cudaStream_t s) {
     const int n_col_ctas = (p.H + kColStrip - 1) / kColStrip;
     const int n_blocks = (p.R + p.block_rows - 1) / p.block_rows;
     const size_t smem = (size_t)n_blocks * kColStrip * sizeof(double);
-    static size_t smem_set = 0;
-    if (smem > 48 * 1024 && smem > smem_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+    static SmemGrant granted;
+    if (smem > 48 * 1024) {
+        cudaError_t e = grant_smem(granted, current_device(), kern, smem);
         if (e != cudaSuccess) return e;
-        smem_set = smem;
     }
     kern<<<n_row_ctas + n_col_ctas, kSmallThreads, smem, s>>>(p);
     return cudaGetLastError();

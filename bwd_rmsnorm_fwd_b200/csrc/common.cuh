@@ -5,6 +5,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "launch_cache.h"
+#include "rmsnorm_train.h"
+
 namespace rmsk {
 
 // A [T, heads, H] row view: row (t, k) starts at element t*st + k*sk.
@@ -69,6 +72,28 @@ constexpr unsigned kStatusTimeout = 1u;
 // default limit of a device-side wait (about two seconds at 2 GHz)
 constexpr int64_t kDefaultWaitCycles = 4000000000LL;
 
+// Raises `kern`'s dynamic shared-memory limit on the current device `dev` to at least
+// `bytes`, once per device (see SmemGrant).
+template <typename K>
+cudaError_t grant_smem(SmemGrant& g, int dev, K kern, size_t bytes) {
+    return static_cast<cudaError_t>(g.grant(dev, (int)bytes, [&](int b) {
+        return (int)cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, b);
+    }));
+}
+
+// Resident CTAs per SM of `kern` at (threads, smem) on device `dev`, cached per device under
+// `key` (at least 1; -1 when the occupancy query fails, with the error in *err).
+template <int N, typename K>
+int resident_ctas(PerDevice<N>& cache, int dev, int key, K kern, int threads, size_t smem,
+                  cudaError_t* err) {
+    return cache.get(dev, key, [&]() {
+        int o = 0;
+        *err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, threads, smem);
+        if (*err != cudaSuccess) return -1;
+        return o > 0 ? o : 1;
+    });
+}
+
 // ---- host-side launchers (defined in fwd.cu / bwd.cu) -------------------------------------
 
 cudaError_t launch_fwd(const FwdParams& p, bool residual, bool w32, cudaStream_t s);
@@ -81,15 +106,26 @@ cudaError_t launch_bwd_nondet(const BwdParams& p, bool residual, bool w32, int g
 // Rows processed together by one CTA of the large backward kernels for this width
 // (the blocks of one deterministic chunk).  Also the chunk's block count.
 int bwd_slots_for_width(int H);
+// The current device (cudaGetDevice; -1 on error) and its SM count (cached per device).
+int current_device();
 int device_sm_count();
 // Fills `maps` for the first n views (box of box_rows rows x H); tensors that cannot use a
 // descriptor get use = 0 and keep the bulk-copy path.
 void make_row_maps(RowMaps* maps, const RowsIn* views, int n, int heads, int H, int64_t rows,
                    int box_rows);
-// Reads and clears the forward's device status word (a library global on the current
-// device); synchronises `s` first.
 // Records `msg` as this thread's rms_last_error() text and returns `code`.
 int set_error(int code, const char* msg);
+
+// Called by the backward entry after every host-side check of a call has passed and just
+// before its first launch; a non-zero return ends the call with that code.
+typedef int (*PreLaunchFn)(void* ctx, cudaStream_t s);
+
+// The backward behind rms_train_bwd / rms_residual_train_bwd (dh == nullptr for the plain
+// form), with an optional hook run right before the launches.
+int bwd_entry(rms_shape shape, rms_rows x, const void* w, int w_dtype, const float* rstd,
+              rms_rows dy, const rms_rows* dh, rms_rows dx, float* dw, int deterministic,
+              void* ws, size_t ws_bytes, int grid_ctas, void* stream, PreLaunchFn hook,
+              void* hook_ctx);
 
 }  // namespace rmsk
 

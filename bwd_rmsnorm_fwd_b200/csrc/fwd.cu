@@ -332,24 +332,13 @@ __global__ void __launch_bounds__(kFwdRowMaxThreads) fwd_row_cta_kernel(const Fw
 
 namespace {
 
-// Resident CTAs per SM of a kernel at a block size (cached per kernel and block size).
-template <typename K>
-int resident_ctas(K kern, int threads, int* cache, size_t smem = 0) {
-    if (*cache == 0) {
-        int o = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, threads, smem) != cudaSuccess)
-            return -1;
-        *cache = o > 0 ? o : 1;
-    }
-    return *cache;
-}
-
 template <int VPT, int ROWS, bool RES, bool W32>
 cudaError_t launch_warp(const FwdParams& p, cudaStream_t s) {
     auto kern = fwd_warp_kernel<VPT, ROWS, RES, W32>;
-    static int occ = 0;
-    const int o = resident_ctas(kern, kFwdWarpThreads, &occ);
-    if (o < 0) return cudaGetLastError();
+    static PerDevice<1> occ;
+    cudaError_t e = cudaSuccess;
+    const int o = resident_ctas(occ, current_device(), 0, kern, kFwdWarpThreads, 0, &e);
+    if (o < 0) return e;
     const int warps_per_cta = kFwdWarpThreads / 32;
     const int64_t groups = ((int64_t)p.R + ROWS - 1) / ROWS;
     const int64_t need = (groups + warps_per_cta - 1) / warps_per_cta;
@@ -380,13 +369,13 @@ template <int VPT, int S, bool RES, bool W32>
 cudaError_t launch_warp_ring(const FwdParams& p, cudaStream_t s) {
     auto kern = fwd_warp_ring_kernel<VPT, S, RES, W32>;
     const size_t smem = (size_t)(kFwdWarpThreads / 32) * S * (RES ? 2 : 1) * VPT * 512;
-    static int occ = 0;
-    if (occ == 0 && smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    const int o = resident_ctas(kern, kFwdWarpThreads, &occ, smem);
-    if (o < 0) return cudaGetLastError();
+    static SmemGrant granted;
+    static PerDevice<1> occ;
+    const int dev = current_device();
+    cudaError_t e = cudaSuccess;
+    if (smem > 48 * 1024 && (e = grant_smem(granted, dev, kern, smem)) != cudaSuccess) return e;
+    const int o = resident_ctas(occ, dev, 0, kern, kFwdWarpThreads, smem, &e);
+    if (o < 0) return e;
     const int64_t need = ((int64_t)p.R + kFwdWarpThreads / 32 - 1) / (kFwdWarpThreads / 32);
     const int64_t cap = (int64_t)device_sm_count() * o;
     const int grid = (int)(need < cap ? need : cap);
@@ -401,19 +390,17 @@ cudaError_t launch_row_cta(const FwdParams& p, cudaStream_t s) {
     const int warps = (p.nvec + 32 * VPT - 1) / (32 * VPT);
     if (warps * 32 > kFwdRowMaxThreads) return cudaErrorInvalidConfiguration;
     const size_t smem = D >= 2 ? (size_t)D * (RES ? 2 : 1) * VPT * warps * 32 * 16 : 0;
+    const int dev = current_device();
+    cudaError_t e = cudaSuccess;
     if constexpr (D >= 2) {
         // the ring of the widest row this instantiation serves (above the 48 KB default)
-        static bool attr = false;
-        if (!attr) {
-            const int most = D * (RES ? 2 : 1) * VPT * kFwdRowMaxThreads * 16;
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
-            if (e != cudaSuccess) return e;
-            attr = true;
-        }
+        static SmemGrant granted;
+        const size_t most = (size_t)D * (RES ? 2 : 1) * VPT * kFwdRowMaxThreads * 16;
+        if ((e = grant_smem(granted, dev, kern, most)) != cudaSuccess) return e;
     }
-    static int occ[kFwdRowMaxThreads / 32 + 1] = {};  // by warp count
-    const int o = resident_ctas(kern, warps * 32, &occ[warps], smem);
-    if (o < 0) return cudaGetLastError();
+    static PerDevice<kFwdRowMaxThreads / 32 + 1> occ;  // by warp count
+    const int o = resident_ctas(occ, dev, warps, kern, warps * 32, smem, &e);
+    if (o < 0) return e;
     const int64_t cap = (int64_t)device_sm_count() * o;
     const int grid = (int)(p.R < cap ? p.R : cap);
     kern<<<grid, warps * 32, smem, s>>>(p);

@@ -96,18 +96,25 @@ int rms_residual_train_fwd(rms_shape shape, rms_rows x, rms_rows residual, const
                            void* stream);
 
 /* Backward.  Reads x (the forward's input), w, rstd (the forward's FP32 output) and dy;
- * writes dx (BF16) and dw (FP32 [H], overwritten, not accumulated).  The workspace
- * (>= rms_train_bwd_workspace_bytes(shape, deterministic, grid_ctas) bytes, 256-byte
- * aligned) must be zero-filled once before its first use; every call leaves it ready
- * for the next.  Calls sharing a workspace must be stream-ordered.  grid_ctas = 0 picks
- * the grid; any other value (1 .. 65535) sets the CTA count of the main backward kernel
- * and never changes the deterministic dw bits.  T == 0 writes dw = 0. */
+ * writes dx (BF16) and dw (FP32 [H], overwritten, not accumulated).  The formulas are
+ * the gradient of the forward (PR #8848 introduction: dx BF16, dw FP32); the two dw
+ * modes are those of the file preamble (deterministic: PR #8512 introduction;
+ * deterministic == 0: PR #8848 introduction and its review on blocked FP32 sums).
+ * The workspace (>= rms_train_bwd_workspace_bytes(shape, deterministic, grid_ctas)
+ * bytes, 256-byte aligned) must be zero-filled once before its first use; every call
+ * leaves it ready for the next.  Calls sharing a workspace must be stream-ordered.
+ * grid_ctas = 0 picks the grid; any other value (1 .. 65535) sets the CTA count of the
+ * main backward kernel and never changes the deterministic dw bits (PR #8512
+ * introduction: dw independent of the grid and the SM count).  T == 0 writes dw = 0. */
 int rms_train_bwd(rms_shape shape, rms_rows x, const void* w, int w_dtype, const float* rstd,
                   rms_rows dy, rms_rows dx, float* dw, int deterministic, void* workspace,
                   size_t workspace_bytes, int grid_ctas, void* stream);
 
-/* Residual backward.  h is the forward's h_out; dy the gradient of y, dh the gradient of
- * h.  Writes grad_h = BF16(dh + dx) and dw.  Workspace rules as rms_train_bwd. */
+/* Residual backward (PR #8512 introduction, "Residual rows": the backward takes the
+ * gradients of y and of h and returns the gradient of h; PR #8848 "Key").  h is the
+ * forward's h_out; dy the gradient of y, dh the gradient of h.  Writes
+ * grad_h = BF16(dh + dx), one rounding of the FP32 sum, and dw.  Workspace rules as
+ * rms_train_bwd. */
 int rms_residual_train_bwd(rms_shape shape, rms_rows h, const void* w, int w_dtype,
                            const float* rstd, rms_rows dy, rms_rows dh, rms_rows grad_h,
                            float* dw, int deterministic, void* workspace,
@@ -121,16 +128,31 @@ int rms_residual_train_bwd(rms_shape shape, rms_rows h, const void* w, int w_dty
  * allocator's callbacks, runtimes that hand out only pre-planned buffers, plugins whose
  * host owns every device buffer -- and so cannot provide a workspace.  The caller still
  * passes every input and output.  H above 8192 is rejected with RMS_EINVAL.  The first
- * call on each device looks up the array's device address (cudaGetSymbolAddress with
- * that device current); make that first call before any stream capture.  Each call
- * clears the scratch it uses on `stream`, and every GPU that loaded the library keeps
- * the array until the process exits.  All calls share the one array, so calls whose
- * work overlaps on the GPU (other streams, unordered threads) race and corrupt dw.
- * Other arguments, checks and outputs are those of rms_train_bwd. */
+ * call on each device (and the first after its context was replaced, e.g. by
+ * cudaDeviceReset) looks up the array's device address (cudaGetSymbolAddress with that
+ * device current); make that first call before any stream capture.  A call that passes
+ * every host-side check clears the ticket and the accumulators it uses on `stream`; a
+ * rejected call queues nothing.  Every GPU that loaded the library keeps the array
+ * until the process exits.  All calls share the one array, so calls whose work overlaps
+ * on the GPU (other streams, unordered threads) race and corrupt dw.  A bounded device
+ * wait that gives up (see rms_set_wait_limit_cycles) leaves the call's outputs invalid
+ * and sets the array's status word, which stays set across later calls until
+ * rms_noalloc_status reads it.  Other arguments, checks and outputs are those of
+ * rms_train_bwd. */
 int rms_train_bwd_noalloc(rms_shape shape, rms_rows x, const void* w, int w_dtype,
                           const float* rstd, rms_rows dy, rms_rows dx, float* dw, void* stream);
 
-/* Workspace bytes the backward needs for this shape, mode and grid (0 on bad input). */
+/* Status of rms_train_bwd_noalloc on the current device (no counterpart on the pages):
+ * synchronises `stream`, then reads and clears the status word of the library's fixed
+ * scratch array.  Returns RMS_OK, RMS_ETIMEOUT (a bounded wait of an earlier call gave up:
+ * that call's dx and dw are invalid) or RMS_ECUDA. */
+int rms_noalloc_status(void* stream);
+
+/* Workspace bytes the backward needs for this shape, mode and grid (0 on bad input).
+ * The workspace holds counters and accumulators only, never rows: a status word, the CTA
+ * ticket, an FP64 accumulator kept zero between calls, and, for the deterministic pair,
+ * the FP64 chunk partials (PR #8512 review summary, "Column-task workspace handling":
+ * counters only, no partial-row capacity). */
 size_t rms_train_bwd_workspace_bytes(rms_shape shape, int deterministic, int grid_ctas);
 
 /* The fixed deterministic summation order for this shape: rows are cut into blocks of
@@ -165,9 +187,10 @@ int64_t rms_set_small_rows_limit(int64_t rows);
 int64_t rms_set_wait_limit_cycles(int64_t cycles);
 
 /* Synchronises `stream` and reads and clears the device status word of `workspace`
- * (written by the backward).  With workspace == NULL it only synchronises: the forward
- * takes no workspace and has no device-side waits, so the stream's own errors are all
- * there is to report.  Returns RMS_OK, RMS_ETIMEOUT or RMS_ECUDA. */
+ * (written by the backward when a bounded device wait gives up; the pages have no
+ * counterpart).  With workspace == NULL it only synchronises: the forward takes no
+ * workspace and has no device-side waits, so the stream's own errors are all there is to
+ * report.  Returns RMS_OK, RMS_ETIMEOUT or RMS_ECUDA. */
 int rms_status(void* workspace, void* stream);
 
 /* Message for the last non-zero return on this thread ("" if none). */

@@ -91,3 +91,69 @@ def test_call_spans_cut_at_the_flush_kernel():
     assert bench.call_spans_us(list(reversed(ev))) == [12.5, 4.0]
     assert bench.call_spans_us([(fill, 0.0, 1.0)]) == []
     assert bench.call_spans_us([("rmsk::k", 2.0, 5.0)]) == [3.0]
+
+
+def _fake_table(n=200):
+    rows = []
+    for i in range(n):
+        rows.append({"cfg": "large-T" if i % 2 else "small-T", "form": "plain", "H": 6144,
+                     "T": 131072, "w": "bf16", "op": ("fwd", "bwd_det", "bwd_nondet")[i % 3],
+                     "us": 700.0 + i, "p10": 690.0, "p90": 720.0, "gbs": 6400.0,
+                     "frac": 0.99 - 0.001 * i, "timer": "cupti_span", "replays": 201,
+                     "replay_us": 705.0, **({"aa_floor": 0.004} if i % 9 == 0 else {})})
+    return rows
+
+
+def test_headline_line_is_last_short_and_complete(tmp_path):
+    """The headline JSON line is the last stdout line, parses, stays under the size limit
+    however long the per-configuration table is (the table goes to its own file), and
+    carries every key of the bench contract."""
+    import io
+    cpu = {"value": 2.2e6, "unit": "us", "cores": 16, "kind": "oracle",
+           "sample": "131072 of 131072 rows of the headline step (fwd, fwd, bwd), 2.2 s",
+           "single_thread": {"value": 3.1e7, "cores": 1, "sample": "9000 of 131072 rows"}}
+    clocks = {"sm_mhz": 1965.0, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"],
+              "samples": 300, "power_w_max": 900.0}
+    line = bench.headline_line(dict(R=bench.HEAD_T, H=bench.HEAD_H, det=False, world=1,
+                                    steps=20, warmup=5, us_step=1790.0, bwd_us=745.0,
+                                    e2e_us=88000.0, peak=6457.1, peak_kind="measured",
+                                    clocks=clocks, cpu=cpu))
+    table = _fake_table()
+    out = io.StringIO()
+    print("some earlier output", file=out)
+    path = tmp_path / "per_config.json"
+    bench.emit(line, table, str(path), 6457.1, "measured", clocks, stream=out)
+    last = out.getvalue().rstrip("\n").splitlines()[-1]
+    assert len(last.encode()) <= bench.MAX_LINE_BYTES
+    d = json.loads(last)
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "roofline", "e2e", "gpu_launches", "clocks", "cpu_baseline"):
+        assert k in d, k
+    assert d["value"] > 0 and d["metric"] == bench.METRIC
+    assert d["config"]["deterministic"] is False and d["config"]["T"] == bench.HEAD_T
+    rf = d["roofline"]
+    assert rf["bound"] == "hbm" and rf["unit"] == "GB/s"
+    assert abs(rf["achieved"] - rf["bytes_per_launch"] / (rf["launch_us"] * 1e-6) / 1e9) < 1.0
+    assert abs(rf["frac"] - rf["achieved"] / rf["peak"]) < 1e-3
+    assert d["e2e"]["h2d_bytes_per_step"] == 2 * bench.HEAD_T * bench.HEAD_H * 2
+    assert d["per_config"]["rows"] == len(table)
+    assert d["per_config"]["large_T_min_frac_fwd"] <= 0.99
+    assert d["per_config"]["aa_floor_max"] == 0.004
+    saved = json.loads(path.read_text())
+    assert len(saved["rows"]) == len(table) and saved["peak_gbs"] == 6457.1
+
+
+def test_oversized_headline_line_is_refused():
+    import io
+    with pytest.raises(RuntimeError):
+        bench.emit({"metric": "x", "blob": "y" * (bench.MAX_LINE_BYTES + 1)}, stream=io.StringIO())
+
+
+def test_interleaved_rounds_rotate_the_order():
+    order = bench.interleaved_order(["a", "b", "c"], rounds=3, reps=2)
+    assert order == ["a", "a", "b", "b", "c", "c",
+                     "b", "b", "c", "c", "a", "a",
+                     "c", "c", "a", "a", "b", "b"]
+    assert len(bench.interleaved_order(list(range(10)), 3, 67)) == 10 * 201
+    assert bench.quantile([1, 2, 3, 4, 5], 0.5) == 3 and bench.quantile([4.0], 0.9) == 4.0
