@@ -2,7 +2,9 @@
 """Benchmark of the training RMSNorm hot path on B200.
 
 Headline workload (one "step"): the checkpointed training step on the large-T
-configuration -- forward, forward recompute, backward (deterministic=False) -- for
+configuration -- forward, forward recompute, backward (deterministic=False), run through
+the library's autograd wrapper under torch.utils.checkpoint, dw added into a float32
+main-grad buffer -- for
 x, dy BF16 [T=131072, H=6144] ~ N(0,1), BF16 weight 1 + 0.1 N(0,1), eps 1e-6, synthetic
 and seeded.  Inputs are far larger than L2 and L2 is also flushed before every timed
 step.  ``value`` is microseconds per step (lower is better); the pages report 1640.48 us
@@ -604,67 +606,75 @@ def main():
     R, H = args.rows, args.width
     x, dy, w = make_inputs(R, H, "bf16", 1234 + rank, dev, torch)
     ws = api.Workspace(dev)
+    # the checkpointed training step through the autograd wrapper: the forward, then the
+    # backward, which recomputes the forward (torch.utils.checkpoint) and runs the library's
+    # backward; dw is added into a float32 main-grad buffer by the accumulate entry point
+    from torch.utils.checkpoint import checkpoint
+    xg = x.detach().requires_grad_(True)
+    main_grad = torch.zeros(H, dtype=torch.float32, device=dev)
 
-    def step():
-        api.rmsnorm_train_fwd(x, w)                       # forward
-        _, rstd = api.rmsnorm_train_fwd(x, w)             # recompute (checkpointed)
-        return rstd
+    def step(x_leaf):
+        x_leaf.grad = None
+        y = checkpoint(api.rmsnorm_train, x_leaf, w, 1e-6, None, args.det, main_grad, ws,
+                       use_reentrant=False)
+        y.backward(dy)
+        return x_leaf.grad
 
     for _ in range(args.warmup):
-        rstd = step()
-        api.rmsnorm_train_bwd(x, w, rstd, dy, deterministic=args.det, workspace=ws)
+        step(xg)
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
     sampler.start()
-    evs = []
+    evs, bwd_evs = [], []
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    for _ in range(args.steps):
-        flush.zero_()
-        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        e0.record()
-        rstd = step()
-        e1.record()
-        api.rmsnorm_train_bwd(x, w, rstd, dy, deterministic=args.det, workspace=ws)
-        e2.record()
-        evs.append((e0, e1, e2))
+    with api.record_backward_events(bwd_evs):
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+            e0.record()
+            step(xg)
+            e1.record()
+            evs.append((e0, e1))
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     clocks = sampler.stop()
     api.status(ws)
-    step_us = [a.elapsed_time(c) * 1e3 for a, b, c in evs]
-    bwd_us = [b.elapsed_time(c) * 1e3 for a, b, c in evs]
+    if len(bwd_evs) != args.steps:
+        raise RuntimeError(f"{len(bwd_evs)} backward calls recorded for {args.steps} steps")
+    step_us = [a.elapsed_time(b) * 1e3 for a, b in evs]
+    bwd_us = [a.elapsed_time(b) * 1e3 for a, b in bwd_evs]
     ms_step = max_over_ranks(sum(step_us) / len(step_us) / 1e3, dist, dev)
     us_step = ms_step * 1e3
     bwd_avg_us = sum(bwd_us) / len(bwd_us)
 
-    # end to end through the public API with pinned host buffers
+    # end to end through the public API (the autograd wrapper) with pinned host buffers: the
+    # step's inputs go in, its results (dx and the accumulated dw) come back, every step
     xh = x.cpu().pin_memory()
     dyh = dy.cpu().pin_memory()
     dxh = torch.empty_like(xh).pin_memory()
     dwh = torch.empty(H, dtype=torch.float32).pin_memory()
     xd = torch.empty_like(x)
-    dyd = torch.empty_like(dy)
     e2e = []
     for i in range(args.e2e_steps + 1 if args.e2e_steps > 0 else 0):
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record()
         xd.copy_(xh, non_blocking=True)
-        dyd.copy_(dyh, non_blocking=True)
-        api.rmsnorm_train_fwd(xd, w)
-        _, r2 = api.rmsnorm_train_fwd(xd, w)
-        dxd, dwd = api.rmsnorm_train_bwd(xd, w, r2, dyd, deterministic=args.det, workspace=ws)
+        dy.copy_(dyh, non_blocking=True)
+        xl = xd.requires_grad_(True)
+        dxd = step(xl)
         dxh.copy_(dxd, non_blocking=True)
-        dwh.copy_(dwd, non_blocking=True)
+        dwh.copy_(main_grad, non_blocking=True)
         b.record()
         b.synchronize()
+        xd = xl.detach()
         if i:
             e2e.append(a.elapsed_time(b) * 1e3)
-    del xd, dyd, xh, dyh, dxh
+    del xd, xh, dyh, dxh, xg
     e2e_us = statistics.median(e2e) if e2e else None
 
     per_cfg = None

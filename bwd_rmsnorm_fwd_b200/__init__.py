@@ -5,8 +5,8 @@ The library is loaded on first use and its absence is an error: there is no CPU 
 eager fallback.
 """
 
-from .api import (Workspace, bwd_path, det_plan, rmsnorm_train_bwd, rmsnorm_train_fwd,
-                  set_small_rows_limit, status)
+from .api import (RMSNormTrainFunction, Workspace, bwd_path, det_plan, rmsnorm_train,
+                  rmsnorm_train_bwd, rmsnorm_train_fwd, set_small_rows_limit, status)
 
-__all__ = ["Workspace", "bwd_path", "det_plan", "rmsnorm_train_bwd", "rmsnorm_train_fwd",
-           "set_small_rows_limit", "status"]
+__all__ = ["RMSNormTrainFunction", "Workspace", "bwd_path", "det_plan", "rmsnorm_train",
+           "rmsnorm_train_bwd", "rmsnorm_train_fwd", "set_small_rows_limit", "status"]

@@ -49,12 +49,23 @@ SIGNATURES = [
     ("rms_residual_train_bwd", _i32,
      [RmsShape, RmsRows, _vp, _i32, _vp, RmsRows, RmsRows, RmsRows, _vp, _i32, _vp, _sz, _i32,
       _vp]),
+    ("rms_train_bwd_accumulate", _i32,
+     [RmsShape, RmsRows, _vp, _i32, _vp, RmsRows, RmsRows, _vp, _i32, _vp, _sz, _i32, _vp]),
+    ("rms_residual_train_bwd_accumulate", _i32,
+     [RmsShape, RmsRows, _vp, _i32, _vp, RmsRows, RmsRows, RmsRows, _vp, _i32, _vp, _sz, _i32,
+      _vp]),
     ("rms_train_bwd_noalloc", _i32,
      [RmsShape, RmsRows, _vp, _i32, _vp, RmsRows, RmsRows, _vp, _vp]),
     ("rms_noalloc_status", _i32, [_vp]),
     ("rms_train_bwd_workspace_bytes", _sz, [RmsShape, _i32, _i32]),
     ("rms_det_plan", _i32, [RmsShape, ctypes.POINTER(ctypes.c_int32),
                             ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),
+    ("rms_det_shard_plan", _i32, [RmsShape, _i32, _i32, ctypes.POINTER(ctypes.c_int64),
+                                  ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_size_t)]),
+    ("rms_train_bwd_det_shard", _i32,
+     [RmsShape, _i32, _i32, RmsRows, _vp, _i32, _vp, RmsRows, RmsRows, RmsRows, _vp, _vp, _sz,
+      _i32, _vp]),
+    ("rms_det_fold_segments", _i32, [RmsShape, _vp, _vp, _i32, _vp]),
     ("rms_train_bwd_path", _i32, [RmsShape, _i32]),
     ("rms_set_small_rows_limit", _i64, [_i64]),
     ("rms_set_wait_limit_cycles", _i64, [_i64]),

@@ -1,6 +1,7 @@
 // C ABI of librmsnorm_train: argument checks, workspace layout, program choice.
 // The declarations and their contract are in include/rmsnorm_train.h.
 #include <atomic>
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -147,6 +148,7 @@ bool use_small(int64_t R, int H) {
 
 struct Plan {
     int32_t B, L, S, n_chunks;
+    int32_t seg_len;  // chunks per fold segment
 };
 
 Plan det_plan(int64_t R, int H) {
@@ -156,10 +158,42 @@ Plan det_plan(int64_t R, int H) {
     p.S = kFoldSegments;
     const int64_t ch = (int64_t)p.B * p.L;
     p.n_chunks = (int32_t)((R + ch - 1) / ch);
+    p.seg_len = (p.n_chunks + p.S - 1) / p.S;
     return p;
 }
 
-size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+// Rows of one rank of a row-sharded deterministic backward: the rank owns 16 / world whole
+// fold segments of the plan of all T rows, so its rows are whole chunks and the folds of
+// its segments are exactly those of the single-GPU order.
+struct ShardPlan {
+    int64_t row_begin, row_end;
+    int32_t n_seg;          // segments of the rank (16 / world)
+    int32_t n_chunks;       // chunks of the rank's rows
+    size_t ws_bytes;
+};
+
+int shard_plan(const rms_shape& s, int rank, int world, ShardPlan* out) {
+    int rc = check_shape(s);
+    if (rc) return rc;
+    if (s.heads != 1)
+        return fail(RMS_EINVAL, "row sharding takes [T, H] rows (heads must be 1, got %d)",
+                    s.heads);
+    if (world < 1 || world > kFoldSegments || kFoldSegments % world)
+        return fail(RMS_EINVAL, "world must divide %d (got %d)", kFoldSegments, world);
+    if (rank < 0 || rank >= world)
+        return fail(RMS_EINVAL, "rank must be in [0, %d) (got %d)", world, rank);
+    const Plan pl = det_plan(s.T, s.H);
+    const int per = kFoldSegments / world;
+    const int64_t c0 = std::min<int64_t>(pl.n_chunks, (int64_t)rank * per * pl.seg_len);
+    const int64_t c1 = std::min<int64_t>(pl.n_chunks, (int64_t)(rank + 1) * per * pl.seg_len);
+    const int64_t ch = (int64_t)pl.B * pl.L;
+    out->row_begin = std::min<int64_t>(s.T, c0 * ch);
+    out->row_end = std::min<int64_t>(s.T, c1 * ch);
+    out->n_seg = per;
+    out->n_chunks = (int32_t)(c1 - c0);
+    out->ws_bytes = kWsHeader + kAccBytes + (size_t)out->n_chunks * s.H * 8;
+    return RMS_OK;
+}
 
 size_t ws_bytes(const rms_shape& s, int det) {
     const int64_t R = s.T * s.heads;
@@ -168,9 +202,26 @@ size_t ws_bytes(const rms_shape& s, int det) {
     return b;
 }
 
+// The workspace: present, 256-byte aligned, at least `need` bytes, apart from every input
+// and output.
+int check_workspace(void* ws, size_t ws_size, size_t need, const Span* ins, int nin,
+                    const Span* outs, int nout) {
+    if (!ws) return fail(RMS_EWORKSPACE, "workspace is null (needs %zu bytes)", need);
+    if (reinterpret_cast<uintptr_t>(ws) % 256)
+        return fail(RMS_EALIGN, "workspace must be 256-byte aligned");
+    if (ws_size < need)
+        return fail(RMS_EWORKSPACE, "workspace has %zu bytes, needs %zu", ws_size, need);
+    const Span wsp = span_of(ws, need, "workspace");
+    for (int i = 0; i < nin; ++i)
+        if (overlap(wsp, ins[i])) return fail(RMS_EALIAS, "workspace overlaps %s", ins[i].name);
+    for (int i = 0; i < nout; ++i)
+        if (overlap(wsp, outs[i])) return fail(RMS_EALIAS, "workspace overlaps %s", outs[i].name);
+    return RMS_OK;
+}
+
 int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const float* rstd,
                rms_rows dy, const rms_rows* dh, rms_rows dx, float* dw, int deterministic,
-               void* ws, size_t ws_size, int grid_ctas, void* stream,
+               void* ws, size_t ws_size, int grid_ctas, void* stream, int accumulate = 0,
                rmsk::PreLaunchFn hook = nullptr, void* hook_ctx = nullptr) {
     int rc = check_shape(shape);
     if (rc) return rc;
@@ -189,6 +240,7 @@ int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const fl
         Span ins[1] = {span_of(w, wb, "w")};
         Span outs[1] = {span_of(dw, (size_t)H * 4, "dw")};
         if ((rc = check_aliases(ins, 1, outs, 1))) return rc;
+        if (accumulate) return ok();  // adding an empty sum leaves dw as it is
         cudaError_t e = cudaMemsetAsync(dw, 0, (size_t)H * 4, st);
         return e == cudaSuccess ? ok() : cuda_fail(e, "cudaMemsetAsync(dw)");
     }
@@ -204,19 +256,8 @@ int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const fl
     if ((rc = check_rows(shape, dx, dh ? "grad_h" : "dx", true, &outs[0]))) return rc;
     outs[1] = span_of(dw, (size_t)H * 4, "dw");
     if ((rc = check_aliases(ins, nin, outs, 2))) return rc;
-    const size_t need = ws_bytes(shape, deterministic);
-    if (!ws) return fail(RMS_EWORKSPACE, "workspace is null (needs %zu bytes)", need);
-    if (reinterpret_cast<uintptr_t>(ws) % 256)
-        return fail(RMS_EALIGN, "workspace must be 256-byte aligned");
-    if (ws_size < need)
-        return fail(RMS_EWORKSPACE, "workspace has %zu bytes, needs %zu", ws_size, need);
-    {
-        Span wsp = span_of(ws, need, "workspace");
-        for (int i = 0; i < nin; ++i)
-            if (overlap(wsp, ins[i])) return fail(RMS_EALIAS, "workspace overlaps %s", ins[i].name);
-        for (int i = 0; i < 2; ++i)
-            if (overlap(wsp, outs[i])) return fail(RMS_EALIAS, "workspace overlaps %s", outs[i].name);
-    }
+    if ((rc = check_workspace(ws, ws_size, ws_bytes(shape, deterministic), ins, nin, outs, 2)))
+        return rc;
 
     rmsk::BwdParams p = {};
     p.R = (int32_t)R;
@@ -240,7 +281,9 @@ int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const fl
     p.blocks_per_chunk = plan.L;
     p.fold_segments = plan.S;
     p.n_chunks = plan.n_chunks;
+    p.seg_len = plan.seg_len;
     p.wait_cycles = g_wait_cycles.load();
+    p.accumulate = accumulate ? 1 : 0;
     const bool res = dh != nullptr;
     const bool w32 = w_dtype == RMS_FP32;
     if (hook && (rc = hook(hook_ctx, st))) return rc;
@@ -253,6 +296,78 @@ int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const fl
         e = rmsk::launch_bwd_nondet(p, res, w32, grid_ctas, st);
     }
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    return ok();
+}
+
+int shard_common(rms_shape shape, int rank, int world, rms_rows x, const void* w, int w_dtype,
+                 const float* rstd, rms_rows dy, rms_rows dh, rms_rows dx, double* seg_out,
+                 void* ws, size_t ws_size, int grid_ctas, void* stream) {
+    ShardPlan sp;
+    int rc = shard_plan(shape, rank, world, &sp);
+    if (rc) return rc;
+    if (w_dtype != RMS_BF16 && w_dtype != RMS_FP32)
+        return fail(RMS_EDTYPE, "w_dtype must be RMS_BF16 or RMS_FP32 (got %d)", w_dtype);
+    if (grid_ctas < 0 || grid_ctas > 65535)
+        return fail(RMS_EINVAL, "grid_ctas must be in [0, 65535] (got %d)", grid_ctas);
+    if (!w || !seg_out) return fail(RMS_EINVAL, "w and seg_out must not be null");
+    if (reinterpret_cast<uintptr_t>(w) % 16 || reinterpret_cast<uintptr_t>(seg_out) % 16)
+        return fail(RMS_EALIGN, "w and seg_out must be 16-byte aligned");
+    const int H = shape.H;
+    const rms_shape local = {sp.row_end - sp.row_begin, 1, H};
+    const int64_t R = local.T;
+    const bool res = dh.ptr != nullptr;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t wb = (size_t)H * (w_dtype == RMS_FP32 ? 4 : 2);
+    const size_t seg_bytes = (size_t)sp.n_seg * H * 8;
+    if (R == 0) {  // a rank whose segments are all empty contributes zeros
+        Span ins[1] = {span_of(w, wb, "w")};
+        Span outs[1] = {span_of(seg_out, seg_bytes, "seg_out")};
+        if ((rc = check_aliases(ins, 1, outs, 1))) return rc;
+        cudaError_t e = cudaMemsetAsync(seg_out, 0, seg_bytes, st);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "cudaMemsetAsync(seg_out)");
+    }
+    if (!rstd) return fail(RMS_EINVAL, "rstd is null");
+    if (reinterpret_cast<uintptr_t>(rstd) % 4) return fail(RMS_EALIGN, "rstd must be 4-byte aligned");
+    Span ins[5], outs[2];
+    int nin = 0;
+    if ((rc = check_rows(local, x, res ? "h" : "x", false, &ins[nin++]))) return rc;
+    if ((rc = check_rows(local, dy, "dy", false, &ins[nin++]))) return rc;
+    if (res && (rc = check_rows(local, dh, "dh", false, &ins[nin++]))) return rc;
+    ins[nin++] = span_of(w, wb, "w");
+    ins[nin++] = span_of(rstd, (size_t)R * 4, "rstd");
+    if ((rc = check_rows(local, dx, res ? "grad_h" : "dx", true, &outs[0]))) return rc;
+    outs[1] = span_of(seg_out, seg_bytes, "seg_out");
+    if ((rc = check_aliases(ins, nin, outs, 2))) return rc;
+    if ((rc = check_workspace(ws, ws_size, sp.ws_bytes, ins, nin, outs, 2))) return rc;
+
+    const Plan plan = det_plan(shape.T, H);  // the order of all rows
+    rmsk::BwdParams p = {};
+    p.R = (int32_t)R;
+    p.heads = 1;
+    p.H = H;
+    p.nvec = H / 8;
+    p.x = in_of(local, x);
+    p.dy = in_of(local, dy);
+    if (res) p.dh = in_of(local, dh);
+    p.dx = out_of(local, dx);
+    p.w = w;
+    p.rstd = rstd;
+    p.dw = nullptr;
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    p.status = reinterpret_cast<unsigned*>(base);
+    p.ticket = reinterpret_cast<unsigned*>(base + 4);
+    p.acc = reinterpret_cast<double*>(base + kWsHeader);
+    p.part = reinterpret_cast<double*>(base + kWsHeader + kAccBytes);
+    p.block_rows = plan.B;
+    p.blocks_per_chunk = plan.L;
+    p.fold_segments = plan.S;
+    p.n_chunks = sp.n_chunks;
+    p.seg_len = plan.seg_len;
+    p.seg_out = seg_out;
+    p.n_seg_out = sp.n_seg;
+    p.wait_cycles = g_wait_cycles.load();
+    cudaError_t e = rmsk::launch_bwd_det(p, res, w_dtype == RMS_FP32, grid_ctas, st);
+    if (e != cudaSuccess) return cuda_fail(e, "sharded backward launch");
     return ok();
 }
 
@@ -270,7 +385,7 @@ int bwd_entry(rms_shape shape, rms_rows x, const void* w, int w_dtype, const flo
               void* ws, size_t ws_bytes, int grid_ctas, void* stream, PreLaunchFn hook,
               void* hook_ctx) {
     return bwd_common(shape, x, w, w_dtype, rstd, dy, dh, dx, dw, deterministic, ws, ws_bytes,
-                      grid_ctas, stream, hook, hook_ctx);
+                      grid_ctas, stream, 0, hook, hook_ctx);
 }
 
 int current_device() {
@@ -374,6 +489,66 @@ int rms_residual_train_bwd(rms_shape shape, rms_rows h, const void* w, int w_dty
                            size_t workspace_bytes, int grid_ctas, void* stream) {
     return bwd_common(shape, h, w, w_dtype, rstd, dy, &dh, grad_h, dw, deterministic, workspace,
                       workspace_bytes, grid_ctas, stream);
+}
+
+int rms_train_bwd_accumulate(rms_shape shape, rms_rows x, const void* w, int w_dtype,
+                             const float* rstd, rms_rows dy, rms_rows dx, float* dw,
+                             int deterministic, void* workspace, size_t workspace_bytes,
+                             int grid_ctas, void* stream) {
+    return bwd_common(shape, x, w, w_dtype, rstd, dy, nullptr, dx, dw, deterministic, workspace,
+                      workspace_bytes, grid_ctas, stream, 1);
+}
+
+int rms_residual_train_bwd_accumulate(rms_shape shape, rms_rows h, const void* w, int w_dtype,
+                                      const float* rstd, rms_rows dy, rms_rows dh,
+                                      rms_rows grad_h, float* dw, int deterministic,
+                                      void* workspace, size_t workspace_bytes, int grid_ctas,
+                                      void* stream) {
+    return bwd_common(shape, h, w, w_dtype, rstd, dy, &dh, grad_h, dw, deterministic, workspace,
+                      workspace_bytes, grid_ctas, stream, 1);
+}
+
+int rms_det_shard_plan(rms_shape shape, int rank, int world, int64_t* row_begin,
+                       int64_t* row_end, size_t* workspace_bytes) {
+    ShardPlan sp;
+    const int rc = shard_plan(shape, rank, world, &sp);
+    if (rc) return rc;
+    if (row_begin) *row_begin = sp.row_begin;
+    if (row_end) *row_end = sp.row_end;
+    if (workspace_bytes) *workspace_bytes = sp.ws_bytes;
+    return ok();
+}
+
+int rms_train_bwd_det_shard(rms_shape shape, int rank, int world, rms_rows x, const void* w,
+                            int w_dtype, const float* rstd, rms_rows dy, rms_rows dh,
+                            rms_rows dx, double* seg_out, void* workspace,
+                            size_t workspace_bytes, int grid_ctas, void* stream) {
+    return shard_common(shape, rank, world, x, w, w_dtype, rstd, dy, dh, dx, seg_out, workspace,
+                        workspace_bytes, grid_ctas, stream);
+}
+
+int rms_det_fold_segments(rms_shape shape, const double* seg, float* dw, int accumulate,
+                          void* stream) {
+    int rc = check_shape(shape);
+    if (rc) return rc;
+    if (!seg || !dw) return fail(RMS_EINVAL, "seg and dw must not be null");
+    if (reinterpret_cast<uintptr_t>(seg) % 16 || reinterpret_cast<uintptr_t>(dw) % 16)
+        return fail(RMS_EALIGN, "seg and dw must be 16-byte aligned");
+    const int H = shape.H;
+    const int64_t R = shape.T * shape.heads;
+    Span ins[1] = {span_of(seg, (size_t)kFoldSegments * H * 8, "seg")};
+    Span outs[1] = {span_of(dw, (size_t)H * 4, "dw")};
+    if ((rc = check_aliases(ins, 1, outs, 1))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (R == 0) {
+        if (accumulate) return ok();
+        cudaError_t e = cudaMemsetAsync(dw, 0, (size_t)H * 4, st);
+        return e == cudaSuccess ? ok() : cuda_fail(e, "cudaMemsetAsync(dw)");
+    }
+    const Plan pl = det_plan(R, H);
+    const int nonempty = (pl.n_chunks + pl.seg_len - 1) / pl.seg_len;
+    cudaError_t e = rmsk::launch_fold_segments(seg, nonempty, H, dw, accumulate, st);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "fold launch");
 }
 
 size_t rms_train_bwd_workspace_bytes(rms_shape shape, int deterministic, int grid_ctas) {

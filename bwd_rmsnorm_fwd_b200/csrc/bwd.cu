@@ -479,8 +479,7 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
         if (*last_flag) {
             __threadfence();
             for (int col = ctid; col < H; col += NCT) {
-                const double a = __ldcg(p.acc + col);
-                p.dw[col] = __double2float_rn(a);
+                store_dw(p, col, __ldcg(p.acc + col));
                 p.acc[col] = 0.0;
             }
             if (ctid == 0) *p.ticket = 0u;
@@ -679,8 +678,7 @@ __global__ void __launch_bounds__(32 * kWarpBwdWarps) bwd_warp_kernel(const BwdP
     if (last) {
         __threadfence();
         for (int col = threadIdx.x; col < H; col += blockDim.x) {
-            const double a = __ldcg(p.acc + col);
-            p.dw[col] = __double2float_rn(a);
+            store_dw(p, col, __ldcg(p.acc + col));
             p.acc[col] = 0.0;
         }
         if (threadIdx.x == 0) *p.ticket = 0u;
@@ -699,9 +697,10 @@ __global__ void __launch_bounds__(32 * kFoldSegMax) bwd_fold_kernel(const BwdPar
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int col = blockIdx.x * 32 + lane;
-    const int nseg = p.fold_segments;
+    const bool shard = p.seg_out != nullptr;
+    const int nseg = shard ? p.n_seg_out : p.fold_segments;
     const int n = p.n_chunks;
-    const int seg_len = (n + nseg - 1) / nseg;
+    const int seg_len = p.seg_len;
     if (warp < nseg && col < p.H) {
         const int k0 = warp * seg_len;
         const int k1 = min(n, k0 + seg_len);
@@ -720,15 +719,32 @@ __global__ void __launch_bounds__(32 * kFoldSegMax) bwd_fold_kernel(const BwdPar
             }
             for (; k < k1; ++k) a += __ldcg(src + (size_t)k * H);
         }
-        seg[warp][lane] = a;
+        if (shard) {
+            p.seg_out[(size_t)warp * p.H + col] = a;  // this shard's segment sums
+        } else {
+            seg[warp][lane] = a;
+        }
     }
+    if (shard) return;
     __syncthreads();
     if (warp == 0 && col < p.H) {
         double tot = seg[0][lane];
         for (int q = 1; q < nseg; ++q)
             if (q * seg_len < n) tot += seg[q][lane];
-        p.dw[col] = __double2float_rn(tot);
+        store_dw(p, col, tot);
     }
+}
+
+// Final fold of a row-sharded deterministic backward: the table of every shard's segment
+// sums, in segment order, folded left to right per column and rounded once.
+__global__ void __launch_bounds__(256) fold_segments_kernel(const double* seg, int n_nonempty,
+                                                            int H, float* dw, int accumulate) {
+    const int col = blockIdx.x * blockDim.x + threadIdx.x;
+    if (col >= H) return;
+    double tot = __ldcg(seg + col);
+    for (int q = 1; q < n_nonempty; ++q) tot += __ldcg(seg + (size_t)q * H + col);
+    const float v = __double2float_rn(tot);
+    dw[col] = accumulate ? __fadd_rn(dw[col], v) : v;
 }
 
 // ============================================================================================
@@ -896,7 +912,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2) bwd_small_kernel(const BwdPa
             }
             tot = (q == 0) ? sg : tot + sg;
         }
-        p.dw[c0 + t] = __double2float_rn(tot);
+        store_dw(p, c0 + t, tot);
     }
 }
 
@@ -1090,6 +1106,12 @@ cudaError_t launch_bwd_det(const BwdParams& p, bool res, bool w32, int grid_ctas
                         : dispatch_large<true, true, false>(p, grid_ctas, s);
     return w32 ? dispatch_large<true, false, true>(p, grid_ctas, s)
                : dispatch_large<true, false, false>(p, grid_ctas, s);
+}
+
+cudaError_t launch_fold_segments(const double* seg, int n_nonempty, int H, float* dw,
+                                 int accumulate, cudaStream_t s) {
+    fold_segments_kernel<<<(H + 255) / 256, 256, 0, s>>>(seg, n_nonempty, H, dw, accumulate);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_nondet(const BwdParams& p, bool res, bool w32, int grid_ctas,

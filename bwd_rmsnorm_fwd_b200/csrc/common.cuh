@@ -55,9 +55,18 @@ struct BwdParams {
     int32_t block_rows;
     int32_t blocks_per_chunk;
     int32_t fold_segments;
-    int32_t n_chunks;
+    int32_t n_chunks;        // chunks of this call's rows
+    int32_t seg_len;         // chunks per fold segment (of the whole problem's plan)
+    // Row-sharded deterministic calls: when non-null the fold kernel writes the FP64 sums
+    // of this shard's n_seg_out segments ([n_seg_out][H]; 0 for an empty segment) instead
+    // of folding them into dw.
+    double* seg_out;
+    int32_t n_seg_out;
     // limit of every device-side wait, in SM clock cycles
     int64_t wait_cycles;
+    // 0: dw = the call's sum; 1: dw = FP32(dw + FP32(the call's sum)), the FP32 sum of the
+    // previous dw and the value the overwrite mode returns
+    int32_t accumulate;
 };
 
 // TMA descriptors of up to three row tensors (x / dy / dh, or x / residual); use[i] != 0
@@ -102,6 +111,10 @@ cudaError_t launch_bwd_det(const BwdParams& p, bool residual, bool w32, int grid
                            cudaStream_t s);
 cudaError_t launch_bwd_nondet(const BwdParams& p, bool residual, bool w32, int grid_ctas,
                               cudaStream_t s);
+// Folds a table of FP64 segment sums seg[n_seg][H] (the first n_nonempty non-empty) left to
+// right per column and rounds once to FP32 into dw (added to dw when accumulate != 0).
+cudaError_t launch_fold_segments(const double* seg, int n_nonempty, int H, float* dw,
+                                 int accumulate, cudaStream_t s);
 
 // Rows processed together by one CTA of the large backward kernels for this width
 // (the blocks of one deterministic chunk).  Also the chunk's block count.
@@ -206,6 +219,12 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
     return __ffma2_rn(b, make_float2(-1.f, -1.f), a);
 }
 __device__ __forceinline__ uint32_t pack2(float2 v) { return pack_bf16x2(v.x, v.y); }
+
+// The one FP32 rounding of a dw column's FP64 total, stored or added to the previous dw.
+__device__ __forceinline__ void store_dw(const BwdParams& p, int col, double total) {
+    const float v = __double2float_rn(total);
+    p.dw[col] = p.accumulate ? __fadd_rn(p.dw[col], v) : v;
+}
 
 __device__ __forceinline__ int64_t row_offset(int32_t r, int32_t heads, int64_t st,
                                               int64_t sk) {

@@ -120,6 +120,24 @@ int rms_residual_train_bwd(rms_shape shape, rms_rows h, const void* w, int w_dty
                            float* dw, int deterministic, void* workspace,
                            size_t workspace_bytes, int grid_ctas, void* stream);
 
+/* Backward with gradient accumulation: rms_train_bwd / rms_residual_train_bwd, except that
+ * dw is read as well as written: dw = FP32(dw + dw_call), where dw_call is exactly what the
+ * overwrite call returns for the same inputs and mode (one FP32 addition of the call's
+ * rounded FP32 sum).  So the deterministic mode's accumulated bits depend only on the
+ * previous dw bits and the inputs.  Used to sum dw over the micro-batches of a step or the
+ * row shards of a batch without a separate add kernel (the pages' checkpointed training
+ * step, PR #8848 "Key", gives the setting; the pages return dw and do not accumulate).
+ * T == 0 leaves dw unchanged.  Other arguments, checks and outputs as the overwrite calls. */
+int rms_train_bwd_accumulate(rms_shape shape, rms_rows x, const void* w, int w_dtype,
+                             const float* rstd, rms_rows dy, rms_rows dx, float* dw,
+                             int deterministic, void* workspace, size_t workspace_bytes,
+                             int grid_ctas, void* stream);
+int rms_residual_train_bwd_accumulate(rms_shape shape, rms_rows h, const void* w, int w_dtype,
+                                      const float* rstd, rms_rows dy, rms_rows dh,
+                                      rms_rows grad_h, float* dw, int deterministic,
+                                      void* workspace, size_t workspace_bytes, int grid_ctas,
+                                      void* stream);
+
 /* Backward without any device allocation: the deterministic == 0 backward of
  * rms_train_bwd, whose scratch (status word, CTA ticket and FP64 accumulators for up to
  * 8192 columns: 65,792 bytes) lives in one fixed device array inside this library
@@ -164,6 +182,37 @@ size_t rms_train_bwd_workspace_bytes(rms_shape shape, int deterministic, int gri
  * Returns RMS_OK or RMS_EINVAL. */
 int rms_det_plan(rms_shape shape, int32_t* block_rows, int32_t* blocks_per_chunk,
                  int32_t* fold_segments);
+
+/* Row-sharded deterministic backward (PR #8512 introduction: the fixed row order, the
+ * fixed-order FP64 fold and the single FP32 rounding, extended across GPUs; the pages run one
+ * GPU).  The T rows of a [T, H] problem (heads == 1) are split over `world` ranks (world
+ * divides 16): rank r owns fold segments [r*16/world, (r+1)*16/world) of the plan of all T
+ * rows (rms_det_plan), which are whole chunks of contiguous rows [row_begin, row_end).
+ * Folding every rank's segment sums in segment order gives dw bit-identical to the
+ * single-GPU deterministic backward of all T rows.
+ *
+ * rms_det_shard_plan: the rows of `rank` and the workspace bytes its shard call needs. */
+int rms_det_shard_plan(rms_shape shape, int rank, int world, int64_t* row_begin,
+                       int64_t* row_end, size_t* workspace_bytes);
+
+/* rms_train_bwd_det_shard: the deterministic backward of rank `rank`'s rows.  `shape` is the
+ * whole problem's [T, 1, H]; x (or h), dy, dh, dx and rstd hold only the rank's
+ * row_end - row_begin rows (views with st = their own row stride).  dh.ptr == NULL selects
+ * the plain form, otherwise the residual form (dx is then grad_h).  Writes dx and, instead
+ * of dw, the FP64 sums of the rank's 16/world segments to seg_out [16/world][H] (16-byte
+ * aligned; 0 for an empty segment).  Workspace as rms_det_shard_plan says, zero-filled once,
+ * as for rms_train_bwd.  The caller gathers every rank's seg_out in rank order into a
+ * [16][H] table (an all-gather; NCCL over NVLink on GPUs) and calls rms_det_fold_segments. */
+int rms_train_bwd_det_shard(rms_shape shape, int rank, int world, rms_rows x, const void* w,
+                            int w_dtype, const float* rstd, rms_rows dy, rms_rows dh,
+                            rms_rows dx, double* seg_out, void* workspace,
+                            size_t workspace_bytes, int grid_ctas, void* stream);
+
+/* rms_det_fold_segments: folds the [16][H] FP64 table of segment sums of the whole problem
+ * `shape` left to right per column (its non-empty segments) and rounds once to FP32 into dw
+ * (dw = FP32(dw + that value) when accumulate != 0).  T == 0 writes dw = 0 (or leaves it). */
+int rms_det_fold_segments(rms_shape shape, const double* seg, float* dw, int accumulate,
+                          void* stream);
 
 /* Which backward program a call with this shape runs: 1 = single-launch small-row
  * kernel (row tasks + column tasks), 2 = main kernel + fixed-order fold kernel
