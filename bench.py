@@ -143,7 +143,7 @@ class ClockSampler:
                 self.samples.append((sm, util, rs, pw))
             except Exception:
                 pass
-            time.sleep(0.02)
+            time.sleep(0.005)
 
     def start(self):
         if self.ok:

@@ -68,6 +68,7 @@ SIGNATURES = [
     ("rms_det_fold_segments", _i32, [RmsShape, _vp, _vp, _i32, _vp]),
     ("rms_train_bwd_path", _i32, [RmsShape, _i32]),
     ("rms_set_small_rows_limit", _i64, [_i64]),
+    ("rms_set_l2_prefetch", _i32, [_i32]),
     ("rms_set_wait_limit_cycles", _i64, [_i64]),
     ("rms_status", _i32, [_vp, _vp]),
     ("rms_last_error", ctypes.c_char_p, []),

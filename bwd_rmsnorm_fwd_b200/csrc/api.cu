@@ -45,6 +45,7 @@ constexpr size_t kAccBytes = (size_t)kMaxH * 8;
 // process-wide settings (rms_set_small_rows_limit, rms_set_wait_limit_cycles)
 std::atomic<int64_t> g_small_rows_override{-1};
 std::atomic<int64_t> g_wait_cycles{rmsk::kDefaultWaitCycles};
+std::atomic<int> g_prefetch{-1};  // -1: the library's choice
 
 struct Span {
     uintptr_t lo, hi;  // [lo, hi)
@@ -138,6 +139,24 @@ int64_t default_small_rows(int H) {
     if (lim > 2048) lim = 2048;
     if (lim < 64) lim = 64;
     return lim;
+}
+
+// L2 prefetch of rows ahead of the pipeline (the pages' mid-size prefetch, PR #8656
+// introduction): rows ahead for the forward's one-CTA-per-row kernel, on/off for the
+// backward's producer.
+int fwd_prefetch(int64_t R, int H) {
+    const int v = g_prefetch.load();
+    if (v >= 0) return v;
+    (void)R;
+    (void)H;
+    return 0;
+}
+int bwd_prefetch(int64_t R, int H) {
+    const int v = g_prefetch.load();
+    if (v >= 0) return v > 0 ? 1 : 0;
+    (void)R;
+    (void)H;
+    return 0;
 }
 
 bool use_small(int64_t R, int H) {
@@ -284,6 +303,7 @@ int bwd_common(rms_shape shape, rms_rows x, const void* w, int w_dtype, const fl
     p.seg_len = plan.seg_len;
     p.wait_cycles = g_wait_cycles.load();
     p.accumulate = accumulate ? 1 : 0;
+    p.prefetch = bwd_prefetch(R, H);
     const bool res = dh != nullptr;
     const bool w32 = w_dtype == RMS_FP32;
     if (hook && (rc = hook(hook_ctx, st))) return rc;
@@ -366,6 +386,7 @@ int shard_common(rms_shape shape, int rank, int world, rms_rows x, const void* w
     p.seg_out = seg_out;
     p.n_seg_out = sp.n_seg;
     p.wait_cycles = g_wait_cycles.load();
+    p.prefetch = bwd_prefetch(R, H);
     cudaError_t e = rmsk::launch_bwd_det(p, res, w_dtype == RMS_FP32, grid_ctas, st);
     if (e != cudaSuccess) return cuda_fail(e, "sharded backward launch");
     return ok();
@@ -436,6 +457,7 @@ int rms_train_fwd(rms_shape shape, rms_rows x, const void* w, int w_dtype, rms_r
     p.w = w;
     p.rstd = rstd;
     p.eps = eps;
+    p.prefetch = fwd_prefetch(R, shape.H);
     cudaError_t e = rmsk::launch_fwd(p, false, w_dtype == RMS_FP32, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "forward launch");
 }
@@ -472,6 +494,7 @@ int rms_residual_train_fwd(rms_shape shape, rms_rows x, rms_rows residual, const
     p.w = w;
     p.rstd = rstd;
     p.eps = eps;
+    p.prefetch = fwd_prefetch(R, shape.H);
     cudaError_t e = rmsk::launch_fwd(p, true, w_dtype == RMS_FP32, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ok() : cuda_fail(e, "residual forward launch");
 }
@@ -578,6 +601,10 @@ int rms_train_bwd_path(rms_shape shape, int deterministic) {
 
 int64_t rms_set_small_rows_limit(int64_t rows) {
     return g_small_rows_override.exchange(rows < 0 ? -1 : rows);
+}
+
+int rms_set_l2_prefetch(int rows) {
+    return g_prefetch.exchange(rows < 0 ? -1 : rows);
 }
 
 int64_t rms_set_wait_limit_cycles(int64_t cycles) {

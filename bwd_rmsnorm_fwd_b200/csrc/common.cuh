@@ -32,6 +32,8 @@ struct FwdParams {
     const void* w;
     float* rstd;
     float eps;
+    // rows ahead of the current one whose inputs are prefetched into L2 (0: none)
+    int32_t prefetch;
 };
 
 struct BwdParams {
@@ -67,6 +69,8 @@ struct BwdParams {
     // 0: dw = the call's sum; 1: dw = FP32(dw + FP32(the call's sum)), the FP32 sum of the
     // previous dw and the value the overwrite mode returns
     int32_t accumulate;
+    // != 0: the producer also prefetches into L2 the rows of the tile one ring ahead
+    int32_t prefetch;
 };
 
 // TMA descriptors of up to three row tensors (x / dy / dh, or x / residual); use[i] != 0
@@ -339,6 +343,12 @@ __device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap* m
         " [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row0), "r"(bar)
         : "memory");
+}
+
+// Bulk prefetch of [src, src + bytes) into L2 (no destination, nothing to wait for); src
+// and bytes must be multiples of 16.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // Bulk copy global -> shared (this CTA), completion counted in bytes on `bar`.

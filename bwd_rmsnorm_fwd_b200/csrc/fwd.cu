@@ -287,8 +287,20 @@ __global__ void __launch_bounds__(kFwdRowMaxThreads) fwd_row_cta_kernel(const Fw
         for (int k = 0; k < D - 1; ++k) issue(k);
     }
     int buf = 0;
+    const uint32_t row_bytes = (uint32_t)p.nvec * 16u;
     for (int k = 0, r = blockIdx.x; r < p.R; ++k, r += G, buf ^= 1) {
         uint4 xv[VPT], rv[RES ? VPT : 1];
+        if (p.prefetch > 0 && t == 0) {
+            // warm L2 with this CTA's next rows (the first time all p.prefetch of them, then
+            // the one that has come into range), one bulk prefetch per row and tensor
+            for (int a = k == 0 ? 1 : p.prefetch; a <= p.prefetch; ++a) {
+                const int rn = r + a * G;
+                if (rn >= p.R) break;
+                prefetch_l2(p.x.ptr + row_offset(rn, p.heads, p.x.st, p.x.sk), row_bytes);
+                if constexpr (RES)
+                    prefetch_l2(p.res.ptr + row_offset(rn, p.heads, p.res.st, p.res.sk), row_bytes);
+            }
+        }
         if constexpr (D >= 2) {
             issue(k + D - 1);
             cp_async_wait<D - 1>();  // this thread's copies of row k have landed

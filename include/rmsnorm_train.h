@@ -226,6 +226,15 @@ int rms_train_bwd_path(rms_shape shape, int deterministic);
  * the default.  Returns the previous override (-1 if none). */
 int64_t rms_set_small_rows_limit(int64_t rows);
 
+/* L2 prefetch of rows ahead of the kernels' own loads (PR #8656 introduction: a bulk L2
+ * prefetch per tensor of the CTA's next row block).  rows > 0: the forward's one-CTA-per-row
+ * kernel (H > 1024) prefetches that many of the CTA's next rows and the backward's
+ * bulk-copy producer prefetches the tile one stage ring ahead; 0 turns both off; -1
+ * restores the library's choice per shape.  Affects later calls in this process (not
+ * thread-safe against concurrent calls); never changes results.  Returns the previous
+ * setting. */
+int rms_set_l2_prefetch(int rows);
+
 /* Limit, in SM clock cycles, of every device-side wait of later launches in this
  * process (the backward's bulk-copy pipeline barrier waits; the forward has none); the
  * default is about two seconds.  A wait that reaches it makes the kernel record
