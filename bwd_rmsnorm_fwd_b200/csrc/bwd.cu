@@ -192,20 +192,6 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                         bulk_load(dst, src.ptr + row_offset(row0, p.heads, src.st, src.sk),
                                   (uint32_t)n * row_bytes, full_bar(stage));
                 }
-                // warm L2 with the rows of the tile that will next use this stage (one bulk
-                // prefetch per tensor and slot; contiguous rows only)
-                if (p.prefetch && t + NS < nt) {
-                    for (int c = lane; c < L * NTEN; c += 32) {
-                        const int ten = c / L;
-                        const int s = c - ten * L;
-                        const RowsIn& src = ten == 0 ? p.x : (ten == 1 ? p.dy : p.dh);
-                        const int row0 = slot_base(u, s) + (t + NS) * P;
-                        const int n = min(P, slot_end(u, s) - row0);
-                        if (n > 0 && rows_contiguous(src, p.heads, H))
-                            prefetch_l2(src.ptr + row_offset(row0, p.heads, src.st, src.sk),
-                                        (uint32_t)n * row_bytes);
-                    }
-                }
                 for (int c = lane; c < RT * NTEN; c += 32) {
                     const int ten = c / RT;
                     const int rr = c - ten * RT;
@@ -767,8 +753,9 @@ __global__ void __launch_bounds__(256) fold_segments_kernel(const double* seg, i
 
 constexpr int kSmallThreads = 512;
 constexpr int kColStrip = 64;   // columns per column task
-constexpr int kRowBatch = 8;    // rows loaded together by a column-task lane (short code:
-                                 // with a cold L2 the instructions come from DRAM too)
+constexpr int kRowBatch = 16;   // rows loaded together by a column-task lane: a whole block
+                                 // of the single-launch regime's order (16 rows), so a block
+                                 // costs one dependent round trip to memory
 
 template <int TPR, int VPT, bool RES, bool W32>
 __global__ void __launch_bounds__(kSmallThreads, 2) bwd_small_kernel(const BwdParams p) {

@@ -69,8 +69,6 @@ struct BwdParams {
     // 0: dw = the call's sum; 1: dw = FP32(dw + FP32(the call's sum)), the FP32 sum of the
     // previous dw and the value the overwrite mode returns
     int32_t accumulate;
-    // != 0: the producer also prefetches into L2 the rows of the tile one ring ahead
-    int32_t prefetch;
 };
 
 // TMA descriptors of up to three row tensors (x / dy / dh, or x / residual); use[i] != 0

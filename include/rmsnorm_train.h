@@ -226,13 +226,12 @@ int rms_train_bwd_path(rms_shape shape, int deterministic);
  * the default.  Returns the previous override (-1 if none). */
 int64_t rms_set_small_rows_limit(int64_t rows);
 
-/* L2 prefetch of rows ahead of the kernels' own loads (PR #8656 introduction: a bulk L2
+/* L2 prefetch of rows ahead of the forward's own loads (PR #8656 introduction: one bulk L2
  * prefetch per tensor of the CTA's next row block).  rows > 0: the forward's one-CTA-per-row
- * kernel (H > 1024) prefetches that many of the CTA's next rows and the backward's
- * bulk-copy producer prefetches the tile one stage ring ahead; 0 turns both off; -1
- * restores the library's choice per shape.  Affects later calls in this process (not
- * thread-safe against concurrent calls); never changes results.  Returns the previous
- * setting. */
+ * kernel (H > 1024) warms that many of the CTA's next rows (x, and the residual); 0 turns it
+ * off; -1 restores the library's choice (one row ahead below 32768 rows, none above, as
+ * measured).  Affects later calls in this process (not thread-safe against concurrent
+ * calls); never changes results.  Returns the previous setting. */
 int rms_set_l2_prefetch(int rows);
 
 /* Limit, in SM clock cycles, of every device-side wait of later launches in this

@@ -16,7 +16,7 @@ import torch
 import oracle
 from bwd_rmsnorm_fwd_b200 import api, synth
 
-from gpu_common import assert_dw, dev_rows, dev_weight, host_bits
+from gpu_common import assert_dw, assert_dx, dev_rows, dev_weight, host_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +42,10 @@ def test_shards_fold_to_the_single_gpu_bits(T, H, wdt, residual, world):
     dhd = dev_rows(dh) if residual else None
     rs = torch.from_numpy(rstd).cuda()
     dx_ref, dw_ref = api.rmsnorm_train_bwd(xd, wd, rs, dyd, deterministic=True, dh=dhd)
+    # the shards run the pipelined pair; where the single-GPU call does too, dx agrees bit
+    # for bit, else (the single-launch program rounds dx its own way) within the dx budget
+    same_program = api.bwd_path(T, 1, H, True) == 2
+    dx_oracle = oracle.train_bwd(x, w, rstd, dy, dh=dh, want_dw=False)[0]
     segs = []
     for rank in range(world):
         b, e, _ = api.shard_rows(T, H, rank, world)
@@ -49,7 +53,9 @@ def test_shards_fold_to_the_single_gpu_bits(T, H, wdt, residual, world):
             xd[b:e], wd, rs[b:e], dyd[b:e], T, rank, world,
             dh=dhd[b:e] if residual else None)
         if e > b:
-            assert np.array_equal(host_bits(dx), host_bits(dx_ref[b:e])), rank
+            if same_program:
+                assert np.array_equal(host_bits(dx), host_bits(dx_ref[b:e])), rank
+            assert_dx(host_bits(dx), dx_oracle[b:e], f"shard dx rank {rank}")
         segs.append(seg)
     table = torch.cat(segs).contiguous()
     dw = api.fold_segments(table, T, H)
