@@ -38,6 +38,68 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Sums of P values over each group of G consecutive lanes at once (G a power of two <= 32,
+// P in {1, 2, 4}, P <= G): a butterfly whose first levels exchange halves of the value set
+// instead of whole values, so P sums cost about as many shuffles as one.  Lane l of a group
+// returns the sum of value q = (l % G) / (G / P).
+template <int G, int P>
+__device__ __forceinline__ float multi_sum(const float (&v)[P], int lane) {
+    static_assert(P == 1 || P == 2 || P == 4, "one, two or four values");
+    static_assert(P <= G && (G & (G - 1)) == 0 && G <= 32, "whole lane groups");
+    constexpr unsigned kAll = 0xFFFFFFFFu;
+    if constexpr (P == 1) {
+        return group_sum<G>(v[0]);
+    } else if constexpr (P == 2) {
+        const bool hi = (lane & (G / 2)) != 0;
+        float a = (hi ? v[1] : v[0]) + __shfl_xor_sync(kAll, hi ? v[0] : v[1], G / 2);
+#pragma unroll
+        for (int o = G / 4; o > 0; o >>= 1) a += __shfl_xor_sync(kAll, a, o);
+        return a;
+    } else {
+        const bool hi = (lane & (G / 2)) != 0;
+        // a0 holds value (hi ? 2 : 0), a1 value (hi ? 3 : 1), each over a lane pair
+        const float a0 = (hi ? v[2] : v[0]) + __shfl_xor_sync(kAll, hi ? v[0] : v[2], G / 2);
+        const float a1 = (hi ? v[3] : v[1]) + __shfl_xor_sync(kAll, hi ? v[1] : v[3], G / 2);
+        const bool mid = (lane & (G / 4)) != 0;
+        float b = (mid ? a1 : a0) + __shfl_xor_sync(kAll, mid ? a0 : a1, G / 4);
+#pragma unroll
+        for (int o = G / 8; o > 0; o >>= 1) b += __shfl_xor_sync(kAll, b, o);
+        return b;
+    }
+}
+
+// The P row dot products of a slot of ST threads (a few lanes of a warp, one warp, or SW
+// warps): every thread passes its partial sums and receives the slot's totals.  Across
+// warps, one partial per (row, warp) meets in the shared buffer `red` ([L][2][P][SW],
+// double-buffered by `buf`) behind the slot's named barrier, and one lane group per row
+// adds them.
+template <int ST, int P>
+__device__ __forceinline__ void slot_dots(const float (&v)[P], float (&dot)[P], float* red,
+                                          int slot, int buf, int lane, int wis) {
+    constexpr unsigned kAll = 0xFFFFFFFFu;
+    constexpr int G = ST < 32 ? ST : 32;
+    constexpr int SW = ST >= 32 ? ST / 32 : 1;
+    constexpr int GP = G / P;  // lanes per row after the butterfly
+    const float mine = multi_sum<G, P>(v, lane);
+    if constexpr (SW == 1) {
+        const int base = lane & ~(G - 1);
+#pragma unroll
+        for (int q = 0; q < P; ++q) dot[q] = __shfl_sync(kAll, mine, base + q * GP);
+    } else {
+        float* r = red + (size_t)(slot * 2 + buf) * P * SW;
+        if (lane % GP == 0) r[(lane / GP) * SW + wis] = mine;
+        named_bar(1 + slot, ST);
+        const int q = lane / GP;
+        float a = 0.f;
+#pragma unroll
+        for (int w = lane % GP; w < SW; w += GP) a += r[q * SW + w];
+#pragma unroll
+        for (int o = GP / 2; o > 0; o >>= 1) a += __shfl_xor_sync(kAll, a, o);
+#pragma unroll
+        for (int qq = 0; qq < P; ++qq) dot[qq] = __shfl_sync(kAll, a, qq * GP);
+    }
+}
+
 // ============================================================================================
 // Large-row kernel: a bulk-copy pipeline.  Warp 0 streams the rows of each tile (x, dy
 // and, in the residual form, dh) into a ring of shared-memory stages with cp.async.bulk,
@@ -66,9 +128,10 @@ struct StagedCfg {
     int32_t stage_offset;
 };
 
-template <int ST, int VPT, int L, int P, bool DET, bool RES, bool W32>
+template <int ST, int VPT, int L, int P, bool DET, bool HOLD, bool RES, bool W32>
 __global__ void __launch_bounds__(32 + ST * L, 1)
     bwd_staged_kernel(const BwdParams p, const StagedCfg sc, const __grid_constant__ RowMaps tm) {
+    static_assert(!HOLD || DET, "only the deterministic consumer holds its rows");
     // ST threads per slot: a few lanes of a warp (8 or 16: several rows per warp), one warp,
     // or several warps (a named barrier joins them)
     static_assert(ST >= 32 ? ST % 32 == 0 : 32 % ST == 0, "slot must tile warps");
@@ -308,8 +371,11 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                                                               (size_t)(slot * P) * row_bytes);
             const uint4* sdh = reinterpret_cast<const uint4*>(sb + 2 * sc.tensor_bytes +
                                                               (size_t)(slot * P) * row_bytes);
-            // pass 1: per-thread partial sums of g * (-xh)
-            float dot[P];
+            // pass 1: per-thread partial sums of g * (-xh).  With HOLD the unpacked -xh and dy
+            // of the tile stay in registers (P rows x VPT vectors) for pass 2, which then
+            // reads no shared memory and unpacks nothing.
+            float dpart[P], dot[P];
+            float2 hx[HOLD ? P : 1][HOLD ? VPT : 1][4], hd[HOLD ? P : 1][HOLD ? VPT : 1][4];
 #pragma unroll
             for (int q = 0; q < P; ++q) {
                 const float2 nrs = make_float2(-rs[q], -rs[q]);
@@ -325,25 +391,25 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const float2 nx = mul2(bf16x2_to_f2(xw[k]), nrs);
-                            const float2 g = mul2(bf16x2_to_f2(dw4[k]), w2[i][k]);
-                            d2 = fma2(g, nx, d2);
+                            const float2 dd = bf16x2_to_f2(dw4[k]);
+                            if constexpr (HOLD) {
+                                hx[q][i][k] = nx;
+                                hd[q][i][k] = dd;
+                            }
+                            d2 = fma2(mul2(dd, w2[i][k]), nx, d2);
+                        }
+                    } else if constexpr (HOLD) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            hx[q][i][k] = make_float2(0.f, 0.f);
+                            hd[q][i][k] = make_float2(0.f, 0.f);
                         }
                     }
                 }
-                dot[q] = group_sum<(ST < 32 ? ST : 32)>(d2.x + d2.y);
+                dpart[q] = d2.x + d2.y;
             }
-            if constexpr (SW > 1) {
-                if (lane == 0) {
-#pragma unroll
-                    for (int q = 0; q < P; ++q) red[((slot * 2 + buf) * P + q) * SW + wis] = dot[q];
-                }
-                named_bar(1 + slot, ST);
-                // every warp re-reduces the SW partials: one shared load and a shuffle tree
-#pragma unroll
-                for (int q = 0; q < P; ++q)
-                    dot[q] = warp_sum(lane < SW ? red[((slot * 2 + buf) * P + q) * SW + lane] : 0.f);
-                buf ^= 1;
-            }
+            slot_dots<ST, P>(dpart, dot, red, slot, buf, lane, wis);
+            if constexpr (SW > 1) buf ^= 1;
             // pass 2: dx = rstd (g - xh c) = rstd (g + nx c), c = -dot / H; dw, rows in order
 #pragma unroll
             for (int q = 0; q < P; ++q) {
@@ -358,10 +424,13 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                 for (int i = 0; i < VPT; ++i) {
                     const int v = ts + ST * i;
                     if (v >= nvec) continue;
-                    const uint4 xr = sx[q * nvec + v];
-                    const uint4 dr = sdy[q * nvec + v];
-                    const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
-                    const uint32_t dw4[4] = {dr.x, dr.y, dr.z, dr.w};
+                    uint32_t xw[4], dw4[4];
+                    if constexpr (!HOLD) {
+                        const uint4 xr = sx[q * nvec + v];
+                        const uint4 dr = sdy[q * nvec + v];
+                        xw[0] = xr.x; xw[1] = xr.y; xw[2] = xr.z; xw[3] = xr.w;
+                        dw4[0] = dr.x; dw4[1] = dr.y; dw4[2] = dr.z; dw4[3] = dr.w;
+                    }
                     uint32_t hw[4] = {0u, 0u, 0u, 0u};
                     if constexpr (RES) {
                         const uint4 hr = sdh[q * nvec + v];
@@ -370,8 +439,14 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                     uint32_t out[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const float2 d = bf16x2_to_f2(dw4[k]);
-                        const float2 nx = mul2(bf16x2_to_f2(xw[k]), nrs);
+                        float2 d, nx;
+                        if constexpr (HOLD) {
+                            d = hd[q][i][k];
+                            nx = hx[q][i][k];
+                        } else {
+                            d = bf16x2_to_f2(dw4[k]);
+                            nx = mul2(bf16x2_to_f2(xw[k]), nrs);
+                        }
                         const float2 g = mul2(d, w2[i][k]);
                         float2 o = mul2(fma2(nx, c2v, g), rs2);
                         if constexpr (RES) o = add2(o, bf16x2_to_f2(hw[k]));
@@ -926,9 +1001,9 @@ namespace {
 
 cudaError_t launch_fold(const BwdParams& p, cudaStream_t s);
 
-template <int ST, int VPT, int L, int P, bool DET, bool RES, bool W32>
+template <int ST, int VPT, int L, int P, bool DET, bool HOLD, bool RES, bool W32>
 cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
-    auto kern = bwd_staged_kernel<ST, VPT, L, P, DET, RES, W32>;
+    auto kern = bwd_staged_kernel<ST, VPT, L, P, DET, HOLD, RES, W32>;
     constexpr int NT = 32 + ST * L;
     constexpr int NTEN = RES ? 3 : 2;
     constexpr size_t kBudget = 220 * 1024;
@@ -1015,15 +1090,40 @@ cudaError_t launch_fold(const BwdParams& p, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, bwd_fold_kernel, p);
 }
 
-// Rows of a slot per stage: 4 when two such stages fit beside the exchange area, else 2.
+// Registers a thread of a warp scheduler may use with one CTA of `warps` warps per SM: each
+// of the 4 schedulers holds 16384 registers and gets ceil(warps / 4) of the warps.
+constexpr int staged_reg_cap(int warps) {
+    return (16384 / (32 * ((warps + 3) / 4))) & ~7;
+}
+
+// Rows per stage of the deterministic consumer that keeps its tile's unpacked rows in
+// registers: it needs about 40 + 24*VPT + 16*VPT*P registers (addresses and row scalars;
+// dw state and weights; the held rows), checked against the per-scheduler cap; 0 where not
+// even two rows fit, and that layout reloads its rows from shared memory in pass 2.
+constexpr int staged_hold_p(int ST, int VPT, int L) {
+    const int cap = staged_reg_cap((32 + ST * L) / 32);
+    const int fixed = 40 + 24 * VPT;
+    return fixed + 64 * VPT <= cap ? 4 : (fixed + 32 * VPT <= cap ? 2 : 0);
+}
+
+// Rows of a slot per stage: the held-row bound of the deterministic consumer above where it
+// holds rows, else 4 when two such stages fit beside the exchange area, else 2.
 template <int ST, int VPT, int L, bool DET, bool RES, bool W32>
 cudaError_t launch_large_p(const BwdParams& p, int grid_ctas, cudaStream_t s) {
+    constexpr int HP = DET ? staged_hold_p(ST, VPT, L) : 0;
     constexpr size_t kRoom = 220 * 1024 - kStagedHeader;
     const size_t xch = (DET && L > 1) ? (size_t)L * p.nvec * 8 * sizeof(double) : 0;
     const size_t row = (size_t)(RES ? 3 : 2) * L * p.H * 2;
-    if (2 * 4 * row + xch + 128 <= kRoom)
-        return launch_large<ST, VPT, L, 4, DET, RES, W32>(p, grid_ctas, s);
-    return launch_large<ST, VPT, L, 2, DET, RES, W32>(p, grid_ctas, s);
+    const bool four = 2 * 4 * row + xch + 128 <= kRoom;
+    if constexpr (HP == 4) {
+        if (four) return launch_large<ST, VPT, L, 4, DET, true, RES, W32>(p, grid_ctas, s);
+        return launch_large<ST, VPT, L, 2, DET, true, RES, W32>(p, grid_ctas, s);
+    } else if constexpr (HP == 2) {
+        return launch_large<ST, VPT, L, 2, DET, true, RES, W32>(p, grid_ctas, s);
+    } else {
+        if (four) return launch_large<ST, VPT, L, 4, DET, false, RES, W32>(p, grid_ctas, s);
+        return launch_large<ST, VPT, L, 2, DET, false, RES, W32>(p, grid_ctas, s);
+    }
 }
 
 // Slot layout per width: ST threads per slot, VPT vectors per thread, L slots per CTA.  L is
