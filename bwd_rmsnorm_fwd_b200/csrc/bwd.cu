@@ -128,10 +128,12 @@ struct StagedCfg {
     int32_t stage_offset;
 };
 
-template <int ST, int VPT, int L, int P, bool DET, bool HOLD, bool RES, bool W32>
+template <int ST, int VPT, int L, int P, bool DET, int NV, bool RES, bool W32>
 __global__ void __launch_bounds__(32 + ST * L, 1)
     bwd_staged_kernel(const BwdParams p, const StagedCfg sc, const __grid_constant__ RowMaps tm) {
-    static_assert(!HOLD || DET, "only the deterministic consumer holds its rows");
+    // NV != 0: the width is exactly NV vectors, every consumer thread owns VPT of them, and
+    // the row size is a compile-time constant (no per-vector range checks, constant offsets)
+    static_assert(NV == 0 || NV == ST * VPT, "a whole-width layout owns every vector");
     // ST threads per slot: a few lanes of a warp (8 or 16: several rows per warp), one warp,
     // or several warps (a named barrier joins them)
     static_assert(ST >= 32 ? ST % 32 == 0 : 32 % ST == 0, "slot must tile warps");
@@ -155,9 +157,9 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
     const int NS = sc.n_stages;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int H = p.H;
-    const int nvec = p.nvec;
-    const uint32_t row_bytes = (uint32_t)H * 2u;
+    const int H = NV ? NV * 8 : p.H;
+    const int nvec = NV ? NV : p.nvec;
+    const uint32_t row_bytes = (uint32_t)nvec * 16u;
     const int64_t limit = p.wait_cycles;
     auto full_bar = [&](int s) { return smem_addr(&bars[s]); };
     auto empty_bar = [&](int s) { return smem_addr(&bars[kMaxStages + s]); };
@@ -303,7 +305,7 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
     for (int i = 0; i < VPT; ++i) {
         const int v = ts + ST * i;
         float wf[8];
-        if (v < nvec) {
+        if (NV || v < nvec) {
             load_w8<W32>(p.w, 8 * v, wf);
         } else {
 #pragma unroll
@@ -371,11 +373,8 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                                                               (size_t)(slot * P) * row_bytes);
             const uint4* sdh = reinterpret_cast<const uint4*>(sb + 2 * sc.tensor_bytes +
                                                               (size_t)(slot * P) * row_bytes);
-            // pass 1: per-thread partial sums of g * (-xh).  With HOLD the unpacked -xh and dy
-            // of the tile stay in registers (P rows x VPT vectors) for pass 2, which then
-            // reads no shared memory and unpacks nothing.
+            // pass 1: per-thread partial sums of g * (-xh)
             float dpart[P], dot[P];
-            float2 hx[HOLD ? P : 1][HOLD ? VPT : 1][4], hd[HOLD ? P : 1][HOLD ? VPT : 1][4];
 #pragma unroll
             for (int q = 0; q < P; ++q) {
                 const float2 nrs = make_float2(-rs[q], -rs[q]);
@@ -383,7 +382,7 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
 #pragma unroll
                 for (int i = 0; i < VPT; ++i) {
                     const int v = ts + ST * i;
-                    if (v < nvec) {
+                    if (NV || v < nvec) {
                         const uint4 xr = sx[q * nvec + v];
                         const uint4 dr = sdy[q * nvec + v];
                         const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
@@ -391,18 +390,7 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const float2 nx = mul2(bf16x2_to_f2(xw[k]), nrs);
-                            const float2 dd = bf16x2_to_f2(dw4[k]);
-                            if constexpr (HOLD) {
-                                hx[q][i][k] = nx;
-                                hd[q][i][k] = dd;
-                            }
-                            d2 = fma2(mul2(dd, w2[i][k]), nx, d2);
-                        }
-                    } else if constexpr (HOLD) {
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            hx[q][i][k] = make_float2(0.f, 0.f);
-                            hd[q][i][k] = make_float2(0.f, 0.f);
+                            d2 = fma2(mul2(bf16x2_to_f2(dw4[k]), w2[i][k]), nx, d2);
                         }
                     }
                 }
@@ -423,14 +411,11 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
 #pragma unroll
                 for (int i = 0; i < VPT; ++i) {
                     const int v = ts + ST * i;
-                    if (v >= nvec) continue;
-                    uint32_t xw[4], dw4[4];
-                    if constexpr (!HOLD) {
-                        const uint4 xr = sx[q * nvec + v];
-                        const uint4 dr = sdy[q * nvec + v];
-                        xw[0] = xr.x; xw[1] = xr.y; xw[2] = xr.z; xw[3] = xr.w;
-                        dw4[0] = dr.x; dw4[1] = dr.y; dw4[2] = dr.z; dw4[3] = dr.w;
-                    }
+                    if (!NV && v >= nvec) continue;
+                    const uint4 xr = sx[q * nvec + v];
+                    const uint4 dr = sdy[q * nvec + v];
+                    const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+                    const uint32_t dw4[4] = {dr.x, dr.y, dr.z, dr.w};
                     uint32_t hw[4] = {0u, 0u, 0u, 0u};
                     if constexpr (RES) {
                         const uint4 hr = sdh[q * nvec + v];
@@ -439,26 +424,23 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                     uint32_t out[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        float2 d, nx;
-                        if constexpr (HOLD) {
-                            d = hd[q][i][k];
-                            nx = hx[q][i][k];
-                        } else {
-                            d = bf16x2_to_f2(dw4[k]);
-                            nx = mul2(bf16x2_to_f2(xw[k]), nrs);
-                        }
+                        const float2 d = bf16x2_to_f2(dw4[k]);
+                        const float2 nx = mul2(bf16x2_to_f2(xw[k]), nrs);
                         const float2 g = mul2(d, w2[i][k]);
                         float2 o = mul2(fma2(nx, c2v, g), rs2);
                         if constexpr (RES) o = add2(o, bf16x2_to_f2(hw[k]));
                         out[k] = pack2(o);
                         if constexpr (DET) {
-                            // -p, its exact error e (fma(-d, -xh, -p) = d xh - p), TwoSum
+                            // -p and its exact error -e = fma(d, -xh, p) (two scalar FMAs with
+                            // a negated addend: cheaper than a packed negation), then TwoSum;
+                            // err + (-e) rounds exactly as err - e
                             const float2 np = mul2(d, nx);
-                            const float2 e = fma2(mul2(d, m1), nx, np);
+                            const float2 ne = make_float2(__fmaf_rn(d.x, nx.x, -np.x),
+                                                          __fmaf_rn(d.y, nx.y, -np.y));
                             const float2 tt = add2(s2[i][k], np);
                             const float2 z = sub2(tt, s2[i][k]);
                             const float2 err = add2(sub2(s2[i][k], sub2(tt, z)), sub2(np, z));
-                            c2[i][k] = add2(c2[i][k], sub2(err, e));
+                            c2[i][k] = add2(c2[i][k], add2(err, ne));
                             s2[i][k] = tt;
                         } else {
                             s2[i][k] = fma2(d, nx, s2[i][k]);
@@ -492,7 +474,7 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
 #pragma unroll
                 for (int i = 0; i < VPT; ++i) {
                     const int v = ts + ST * i;
-                    if (v >= nvec) continue;
+                    if (!NV && v >= nvec) continue;
                     double* dst = p.part + (size_t)k * H + 8 * v;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
@@ -507,7 +489,7 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
 #pragma unroll
                     for (int i = 0; i < VPT; ++i) {
                         const int v = ts + ST * i;
-                        if (v >= nvec) continue;
+                        if (!NV && v >= nvec) continue;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             my64[8 * v + 2 * kk] = -((double)s2[i][kk].x + (double)c2[i][kk].x);
@@ -536,7 +518,7 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int v = ts + ST * i;
-            if (v >= nvec) continue;
+            if (!NV && v >= nvec) continue;
 #pragma unroll
             for (int e = 0; e < 8; ++e) tot[(size_t)slot * nvec * 8 + 8 * v + e] = acc[i][e];
         }
@@ -1001,9 +983,9 @@ namespace {
 
 cudaError_t launch_fold(const BwdParams& p, cudaStream_t s);
 
-template <int ST, int VPT, int L, int P, bool DET, bool HOLD, bool RES, bool W32>
+template <int ST, int VPT, int L, int P, bool DET, int NV, bool RES, bool W32>
 cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
-    auto kern = bwd_staged_kernel<ST, VPT, L, P, DET, HOLD, RES, W32>;
+    auto kern = bwd_staged_kernel<ST, VPT, L, P, DET, NV, RES, W32>;
     constexpr int NT = 32 + ST * L;
     constexpr int NTEN = RES ? 3 : 2;
     constexpr size_t kBudget = 220 * 1024;
@@ -1090,40 +1072,27 @@ cudaError_t launch_fold(const BwdParams& p, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, bwd_fold_kernel, p);
 }
 
-// Registers a thread of a warp scheduler may use with one CTA of `warps` warps per SM: each
-// of the 4 schedulers holds 16384 registers and gets ceil(warps / 4) of the warps.
-constexpr int staged_reg_cap(int warps) {
-    return (16384 / (32 * ((warps + 3) / 4))) & ~7;
+// Rows of a slot per stage: 4 when two such stages fit beside the exchange area, else 2;
+// the whole-width instantiation when the row is exactly ST*VPT vectors and a slot has at
+// least two warps (with fewer threads per row the compiler hoists a whole tile's loads
+// once the offsets are constant, and spills).
+template <int ST, int VPT, int L, int P, bool DET, bool RES, bool W32>
+cudaError_t launch_large_nv(const BwdParams& p, int grid_ctas, cudaStream_t s) {
+    if constexpr (ST >= 64) {
+        if (p.nvec == ST * VPT)
+            return launch_large<ST, VPT, L, P, DET, ST * VPT, RES, W32>(p, grid_ctas, s);
+    }
+    return launch_large<ST, VPT, L, P, DET, 0, RES, W32>(p, grid_ctas, s);
 }
 
-// Rows per stage of the deterministic consumer that keeps its tile's unpacked rows in
-// registers: it needs about 40 + 24*VPT + 16*VPT*P registers (addresses and row scalars;
-// dw state and weights; the held rows), checked against the per-scheduler cap; 0 where not
-// even two rows fit, and that layout reloads its rows from shared memory in pass 2.
-constexpr int staged_hold_p(int ST, int VPT, int L) {
-    const int cap = staged_reg_cap((32 + ST * L) / 32);
-    const int fixed = 40 + 24 * VPT;
-    return fixed + 64 * VPT <= cap ? 4 : (fixed + 32 * VPT <= cap ? 2 : 0);
-}
-
-// Rows of a slot per stage: the held-row bound of the deterministic consumer above where it
-// holds rows, else 4 when two such stages fit beside the exchange area, else 2.
 template <int ST, int VPT, int L, bool DET, bool RES, bool W32>
 cudaError_t launch_large_p(const BwdParams& p, int grid_ctas, cudaStream_t s) {
-    constexpr int HP = DET ? staged_hold_p(ST, VPT, L) : 0;
     constexpr size_t kRoom = 220 * 1024 - kStagedHeader;
     const size_t xch = (DET && L > 1) ? (size_t)L * p.nvec * 8 * sizeof(double) : 0;
     const size_t row = (size_t)(RES ? 3 : 2) * L * p.H * 2;
-    const bool four = 2 * 4 * row + xch + 128 <= kRoom;
-    if constexpr (HP == 4) {
-        if (four) return launch_large<ST, VPT, L, 4, DET, true, RES, W32>(p, grid_ctas, s);
-        return launch_large<ST, VPT, L, 2, DET, true, RES, W32>(p, grid_ctas, s);
-    } else if constexpr (HP == 2) {
-        return launch_large<ST, VPT, L, 2, DET, true, RES, W32>(p, grid_ctas, s);
-    } else {
-        if (four) return launch_large<ST, VPT, L, 4, DET, false, RES, W32>(p, grid_ctas, s);
-        return launch_large<ST, VPT, L, 2, DET, false, RES, W32>(p, grid_ctas, s);
-    }
+    if (2 * 4 * row + xch + 128 <= kRoom)
+        return launch_large_nv<ST, VPT, L, 4, DET, RES, W32>(p, grid_ctas, s);
+    return launch_large_nv<ST, VPT, L, 2, DET, RES, W32>(p, grid_ctas, s);
 }
 
 // Slot layout per width: ST threads per slot, VPT vectors per thread, L slots per CTA.  L is
