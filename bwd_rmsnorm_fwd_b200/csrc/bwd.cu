@@ -68,6 +68,29 @@ __device__ __forceinline__ float multi_sum(const float (&v)[P], int lane) {
     }
 }
 
+// The P row dot products of a slot of ST threads, one row at a time: a shuffle tree per row,
+// then (slots of several warps) one partial per (row, warp) behind the slot's named barrier
+// and a second tree over them.  Measured faster than slot_dots for the blocked-FP32 consumer
+// of multi-warp slots, where its per-row trees interleave with the rest of the pass.
+template <int ST, int P>
+__device__ __forceinline__ void slot_dots_rowwise(const float (&v)[P], float (&dot)[P], float* red,
+                                                  int slot, int buf, int lane, int wis) {
+    constexpr int G = ST < 32 ? ST : 32;
+    constexpr int SW = ST >= 32 ? ST / 32 : 1;
+#pragma unroll
+    for (int q = 0; q < P; ++q) dot[q] = group_sum<G>(v[q]);
+    if constexpr (SW > 1) {
+        float* r = red + (size_t)(slot * 2 + buf) * P * SW;
+        if (lane == 0) {
+#pragma unroll
+            for (int q = 0; q < P; ++q) r[q * SW + wis] = dot[q];
+        }
+        named_bar(1 + slot, ST);
+#pragma unroll
+        for (int q = 0; q < P; ++q) dot[q] = warp_sum(lane < SW ? r[q * SW + lane] : 0.f);
+    }
+}
+
 // The P row dot products of a slot of ST threads (a few lanes of a warp, one warp, or SW
 // warps): every thread passes its partial sums and receives the slot's totals.  Across
 // warps, one partial per (row, warp) meets in the shared buffer `red` ([L][2][P][SW],
@@ -396,7 +419,10 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                 }
                 dpart[q] = d2.x + d2.y;
             }
-            slot_dots<ST, P>(dpart, dot, red, slot, buf, lane, wis);
+            if constexpr (DET || SW == 1)
+                slot_dots<ST, P>(dpart, dot, red, slot, buf, lane, wis);
+            else
+                slot_dots_rowwise<ST, P>(dpart, dot, red, slot, buf, lane, wis);
             if constexpr (SW > 1) buf ^= 1;
             // pass 2: dx = rstd (g - xh c) = rstd (g + nx c), c = -dot / H; dw, rows in order
 #pragma unroll
@@ -1072,13 +1098,14 @@ cudaError_t launch_fold(const BwdParams& p, cudaStream_t s) {
     return cudaLaunchKernelEx(&cfg, bwd_fold_kernel, p);
 }
 
-// Rows of a slot per stage: 4 when two such stages fit beside the exchange area, else 2;
-// the whole-width instantiation when the row is exactly ST*VPT vectors and a slot has at
-// least two warps (with fewer threads per row the compiler hoists a whole tile's loads
-// once the offsets are constant, and spills).
+// Rows of a slot per stage: 4 when two such stages fit beside the exchange area, else 2.
+// The deterministic consumer gets the whole-width instantiation when the row is exactly
+// ST*VPT vectors and a slot has at least two warps (measured 4-16 % faster at H 1536-6144;
+// with fewer threads per row the compiler hoists a whole tile's loads once the offsets are
+// constant, and spills; the blocked-FP32 consumer measured slower with it).
 template <int ST, int VPT, int L, int P, bool DET, bool RES, bool W32>
 cudaError_t launch_large_nv(const BwdParams& p, int grid_ctas, cudaStream_t s) {
-    if constexpr (ST >= 64) {
+    if constexpr (DET && ST >= 64) {
         if (p.nvec == ST * VPT)
             return launch_large<ST, VPT, L, P, DET, ST * VPT, RES, W32>(p, grid_ctas, s);
     }
