@@ -71,7 +71,7 @@ __device__ __forceinline__ float multi_sum(const float (&v)[P], int lane) {
 // The P row dot products of a slot of ST threads, one row at a time: a shuffle tree per row,
 // then (slots of several warps) one partial per (row, warp) behind the slot's named barrier
 // and a second tree over them.  Measured faster than slot_dots for the blocked-FP32 consumer
-// of multi-warp slots, where its per-row trees interleave with the rest of the pass.
+// when one multi-warp slot fills the CTA.
 template <int ST, int P>
 __device__ __forceinline__ void slot_dots_rowwise(const float (&v)[P], float (&dot)[P], float* red,
                                                   int slot, int buf, int lane, int wis) {
@@ -147,7 +147,7 @@ struct StagedCfg {
     int32_t n_stages;
     int32_t stage_bytes;   // one stage, all tensors
     int32_t tensor_bytes;  // one tensor's rows inside a stage
-    int32_t xch_offset;    // FP64 [L][nvec*8] exchange / accumulators
+    int32_t xch_offset;    // FP64 [nvec*8] running sum of a chunk's blocks
     int32_t stage_offset;
 };
 
@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 16 * kMaxStages);
     volatile unsigned* last_flag = reinterpret_cast<volatile unsigned*>(smem + 16 * kMaxStages + 4);
     float* red = reinterpret_cast<float*>(smem + 16 * kMaxStages + 16);  // [L][2][P][SW]
-    double* xch = reinterpret_cast<double*>(smem + sc.xch_offset);       // [L][nvec*8]
+    double* xch = reinterpret_cast<double*>(smem + sc.xch_offset);       // [nvec*8] running chunk sum
     unsigned char* stages = smem + sc.stage_offset;
 
     const int NS = sc.n_stages;
@@ -320,7 +320,6 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
     const int ts = ctid - slot * ST;
     const int wis = ts >> 5;
     const float invH = 1.0f / (float)H;
-    double* my64 = xch + (size_t)slot * nvec * 8;
     const float2 m1 = make_float2(-1.f, -1.f);
 
     float2 w2[VPT][4];
@@ -419,7 +418,10 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                 }
                 dpart[q] = d2.x + d2.y;
             }
-            if constexpr (DET || SW == 1)
+            // the blocked-FP32 consumer of one multi-warp slot per CTA reduces row by row
+            // (measured faster there: H 4096-6144); every other layout takes the multi-row
+            // butterfly (H 2048 blocked FP32 with two slots: 137 vs 162 us)
+            if constexpr (DET || SW == 1 || L > 1)
                 slot_dots<ST, P>(dpart, dot, red, slot, buf, lane, wis);
             else
                 slot_dots_rowwise<ST, P>(dpart, dot, red, slot, buf, lane, wis);
@@ -511,25 +513,37 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                     }
                 }
             } else {
-                if (slot < nb) {
+                // the chunk's blocks folded left to right through one FP64 row: slot b adds
+                // its block to the running sum after slot b - 1 has (one consumer barrier per
+                // block), and the last block's slot stores the chunk partial
+                for (int b = 0; b < nb; ++b) {
+                    if (slot == b) {
 #pragma unroll
-                    for (int i = 0; i < VPT; ++i) {
-                        const int v = ts + ST * i;
-                        if (!NV && v >= nvec) continue;
+                        for (int i = 0; i < VPT; ++i) {
+                            const int v = ts + ST * i;
+                            if (!NV && v >= nvec) continue;
+                            double* run = xch + 8 * v;
+                            double* dst = p.part + (size_t)k * H + 8 * v;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            my64[8 * v + 2 * kk] = -((double)s2[i][kk].x + (double)c2[i][kk].x);
-                            my64[8 * v + 2 * kk + 1] = -((double)s2[i][kk].y + (double)c2[i][kk].y);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                double2 t2;
+                                t2.x = -((double)s2[i][kk].x + (double)c2[i][kk].x);
+                                t2.y = -((double)s2[i][kk].y + (double)c2[i][kk].y);
+                                if (b > 0) {
+                                    t2.x = run[2 * kk] + t2.x;
+                                    t2.y = run[2 * kk + 1] + t2.y;
+                                }
+                                if (b + 1 < nb) {
+                                    run[2 * kk] = t2.x;
+                                    run[2 * kk + 1] = t2.y;
+                                } else {
+                                    *reinterpret_cast<double2*>(dst + 2 * kk) = t2;
+                                }
+                            }
                         }
                     }
+                    named_bar(kAllConsumers, NCT);
                 }
-                named_bar(kAllConsumers, NCT);
-                for (int col = ctid; col < H; col += NCT) {
-                    double a = xch[col];
-                    for (int b = 1; b < nb; ++b) a += xch[(size_t)b * nvec * 8 + col];
-                    p.part[(size_t)k * H + col] = a;
-                }
-                named_bar(kAllConsumers, NCT);
             }
         }
     }
@@ -1016,7 +1030,7 @@ cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     constexpr int NTEN = RES ? 3 : 2;
     constexpr size_t kBudget = 220 * 1024;
     StagedCfg sc;
-    const size_t xch = (DET && L > 1) ? (size_t)L * p.nvec * 8 * sizeof(double) : 0;
+    const size_t xch = (DET && L > 1) ? (size_t)p.nvec * 8 * sizeof(double) : 0;
     sc.xch_offset = kStagedHeader;
     sc.stage_offset = (int32_t)(kStagedHeader + ((xch + 127) & ~size_t(127)));
     sc.tensor_bytes = L * P * p.H * 2;
@@ -1115,7 +1129,7 @@ cudaError_t launch_large_nv(const BwdParams& p, int grid_ctas, cudaStream_t s) {
 template <int ST, int VPT, int L, bool DET, bool RES, bool W32>
 cudaError_t launch_large_p(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     constexpr size_t kRoom = 220 * 1024 - kStagedHeader;
-    const size_t xch = (DET && L > 1) ? (size_t)L * p.nvec * 8 * sizeof(double) : 0;
+    const size_t xch = (DET && L > 1) ? (size_t)p.nvec * 8 * sizeof(double) : 0;
     const size_t row = (size_t)(RES ? 3 : 2) * L * p.H * 2;
     if (2 * 4 * row + xch + 128 <= kRoom)
         return launch_large_nv<ST, VPT, L, 4, DET, RES, W32>(p, grid_ctas, s);
@@ -1133,6 +1147,12 @@ cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     if constexpr (!DET) {
         if (nv <= 64 && (int64_t)p.R * p.H < kWarpBwdMaxElems)
             return dispatch_warp_bwd<RES, W32>(p, grid_ctas, s);
+    }
+    if constexpr (DET) {
+        // thinner slots for the narrowest rows: twice the consumer warps (measured: H 512 x
+        // 131072 100 vs 105 us, [16384,24,256] 156 vs 161 us); same L, so the same order
+        if (nv <= 32) return launch_large_p<32, 1, 16, DET, RES, W32>(p, grid_ctas, s);
+        if (nv <= 64) return launch_large_p<64, 1, 8, DET, RES, W32>(p, grid_ctas, s);
     }
     if (nv <= 32) return launch_large_p<16, 2, 16, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 64) return launch_large_p<32, 2, 8, DET, RES, W32>(p, grid_ctas, s);

@@ -252,7 +252,7 @@ __device__ __forceinline__ void load_row(const FwdParams& p, int r, uint4 (&xv)[
     }
 }
 
-template <int VPT, int D, bool RES, bool W32>
+template <int VPT, int D, bool RES, bool W32, bool PF>
 __global__ void __launch_bounds__(kFwdRowMaxThreads) fwd_row_cta_kernel(const FwdParams p) {
     constexpr int NTEN = RES ? 2 : 1;
     __shared__ float red[2][kFwdRowMaxThreads / 32];
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kFwdRowMaxThreads) fwd_row_cta_kernel(const Fw
     const uint32_t row_bytes = (uint32_t)p.nvec * 16u;
     for (int k = 0, r = blockIdx.x; r < p.R; ++k, r += G, buf ^= 1) {
         uint4 xv[VPT], rv[RES ? VPT : 1];
-        if (p.prefetch > 0 && t == 0) {
+        if (PF && t == 0) {
             // warm L2 with this CTA's next rows (the first time all p.prefetch of them, then
             // the one that has come into range), one bulk prefetch per row and tensor
             for (int a = k == 0 ? 1 : p.prefetch; a <= p.prefetch; ++a) {
@@ -395,10 +395,15 @@ cudaError_t launch_warp_ring(const FwdParams& p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-// One CTA per row: ceil(nvec / (32 VPT)) warps; a D-row cp.async ring when D >= 2.
-template <int VPT, int D, bool RES, bool W32>
+// One CTA per row: ceil(nvec / (32 VPT)) warps; a D-row cp.async ring when D >= 2.  PF: the
+// L2 prefetch of the CTA's next rows is compiled in (its registers would cost resident CTAs
+// where it is off: 40 -> 44 registers, 12 -> 10 CTAs per SM at H 2048, FP32 weight).
+template <int VPT, int D, bool RES, bool W32, bool PF = false>
 cudaError_t launch_row_cta(const FwdParams& p, cudaStream_t s) {
-    auto kern = fwd_row_cta_kernel<VPT, D, RES, W32>;
+    if constexpr (!PF && D == 0) {
+        if (p.prefetch > 0) return launch_row_cta<VPT, D, RES, W32, true>(p, s);
+    }
+    auto kern = fwd_row_cta_kernel<VPT, D, RES, W32, PF>;
     const int warps = (p.nvec + 32 * VPT - 1) / (32 * VPT);
     if (warps * 32 > kFwdRowMaxThreads) return cudaErrorInvalidConfiguration;
     const size_t smem = D >= 2 ? (size_t)D * (RES ? 2 : 1) * VPT * warps * 32 * 16 : 0;
