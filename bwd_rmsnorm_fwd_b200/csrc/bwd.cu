@@ -395,11 +395,12 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                                                               (size_t)(slot * P) * row_bytes);
             const uint4* sdh = reinterpret_cast<const uint4*>(sb + 2 * sc.tensor_bytes +
                                                               (size_t)(slot * P) * row_bytes);
-            // pass 1: per-thread partial sums of g * (-xh)
+            // pass 1: per-thread partial sums of g * x, scaled by -rstd once per row to give
+            // the partial sums of g * (-xh) (one packed multiply per pair fewer than forming
+            // -xh here; the dot only enters dx)
             float dpart[P], dot[P];
 #pragma unroll
             for (int q = 0; q < P; ++q) {
-                const float2 nrs = make_float2(-rs[q], -rs[q]);
                 float2 d2 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int i = 0; i < VPT; ++i) {
@@ -410,13 +411,11 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                         const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
                         const uint32_t dw4[4] = {dr.x, dr.y, dr.z, dr.w};
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const float2 nx = mul2(bf16x2_to_f2(xw[k]), nrs);
-                            d2 = fma2(mul2(bf16x2_to_f2(dw4[k]), w2[i][k]), nx, d2);
-                        }
+                        for (int k = 0; k < 4; ++k)
+                            d2 = fma2(mul2(bf16x2_to_f2(dw4[k]), w2[i][k]), bf16x2_to_f2(xw[k]), d2);
                     }
                 }
-                dpart[q] = d2.x + d2.y;
+                dpart[q] = (d2.x + d2.y) * -rs[q];
             }
             // the blocked-FP32 consumer of one multi-warp slot per CTA reduces row by row
             // (measured faster there: H 4096-6144); every other layout takes the multi-row
@@ -850,9 +849,9 @@ __global__ void __launch_bounds__(256) fold_segments_kernel(const double* seg, i
 
 constexpr int kSmallThreads = 512;
 constexpr int kColStrip = 64;   // columns per column task
-constexpr int kRowBatch = 16;   // rows loaded together by a column-task lane: a whole block
-                                 // of the single-launch regime's order (16 rows), so a block
-                                 // costs one dependent round trip to memory
+constexpr int kRowBatch = 8;    // rows loaded together by a column-task lane (short code:
+                                 // with a cold L2 the instructions come from DRAM too; loading
+                                 // a whole 16-row block at once measured 1-1.5 us slower)
 
 template <int TPR, int VPT, bool RES, bool W32>
 __global__ void __launch_bounds__(kSmallThreads, 2) bwd_small_kernel(const BwdParams p) {
