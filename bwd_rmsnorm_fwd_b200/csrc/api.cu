@@ -120,13 +120,17 @@ rmsk::RowsOut out_of(const rms_shape& s, const rms_rows& v) {
 
 // ---- the deterministic order and the program choice --------------------------------------
 
-// Rows per block of the deterministic order: 16 in the single-launch regime, otherwise the
-// largest power of two in [8, 64] that still cuts the rows into at least kMinChunks chunks of
-// L blocks (one per SM of a B200), so mid-sized problems keep every SM busy.  A function of
-// (R, L) -- that is, of the row count and the width -- and of nothing else.
+// Rows per block of the deterministic order: in the single-launch regime 8 up to 128 rows
+// (at most 16 blocks: each warp of a column task sums one block after one round of loads;
+// measured 1-1.5 us faster at T 32-87) and 16 up to 2048 rows (8-row blocks there give a warp
+// two blocks and measured slower at T 227); otherwise the largest power of two in [8, 64]
+// that still cuts the rows into at least kMinChunks chunks of L blocks (one per SM of a
+// B200), so mid-sized problems keep every SM busy.  A function of (R, L) -- that is, of the
+// row count and the width -- and of nothing else.
 constexpr int64_t kMinChunks = 148;
 
 int32_t det_block_rows(int64_t R, int L) {
+    if (R <= 128) return 8;
     if (R <= 2048) return 16;
     int32_t B = 64;
     while (B > 8 && (R + (int64_t)B * L - 1) / ((int64_t)B * L) < kMinChunks) B /= 2;

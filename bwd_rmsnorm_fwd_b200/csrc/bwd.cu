@@ -849,9 +849,9 @@ __global__ void __launch_bounds__(256) fold_segments_kernel(const double* seg, i
 
 constexpr int kSmallThreads = 512;
 constexpr int kColStrip = 64;   // columns per column task
-constexpr int kRowBatch = 8;    // rows loaded together by a column-task lane (short code:
-                                 // with a cold L2 the instructions come from DRAM too; loading
-                                 // a whole 16-row block at once measured 1-1.5 us slower)
+constexpr int kRowBatch = 8;    // rows loaded together by a column-task lane: one block of the
+                                 // single-launch regime's order (short code: with a cold L2 the
+                                 // instructions come from DRAM too)
 
 template <int TPR, int VPT, bool RES, bool W32>
 __global__ void __launch_bounds__(kSmallThreads, 2) bwd_small_kernel(const BwdParams p) {
@@ -1140,6 +1140,8 @@ cudaError_t launch_large_p(const BwdParams& p, int grid_ctas, cudaStream_t s) {
 // bwd_slots_for_width); ST and VPT are free and were measured per width and mode: narrow rows
 // share a warp between rows, and the deterministic mode, which carries a TwoSum state per
 // column, runs best with more threads and fewer columns per thread.
+constexpr int kThinDetRows = 131072;
+
 template <bool DET, bool RES, bool W32>
 cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     const int nv = p.nvec;
@@ -1148,10 +1150,13 @@ cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
             return dispatch_warp_bwd<RES, W32>(p, grid_ctas, s);
     }
     if constexpr (DET) {
-        // thinner slots for the narrowest rows: twice the consumer warps (measured: H 512 x
-        // 131072 100 vs 105 us, [16384,24,256] 156 vs 161 us); same L, so the same order
-        if (nv <= 32) return launch_large_p<32, 1, 16, DET, RES, W32>(p, grid_ctas, s);
-        if (nv <= 64) return launch_large_p<64, 1, 8, DET, RES, W32>(p, grid_ctas, s);
+        // thinner slots for the narrowest rows at many rows: twice the consumer warps
+        // (measured: H 512 x 131072 100 vs 105 us, [16384,24,256] 156 vs 161 us; slower below:
+        // [1024,24,256] 28.9 vs 25.1 us, [16384,4,256] 39.8 vs 38.6 us); same L, same order
+        if (p.R >= kThinDetRows) {
+            if (nv <= 32) return launch_large_p<32, 1, 16, DET, RES, W32>(p, grid_ctas, s);
+            if (nv <= 64) return launch_large_p<64, 1, 8, DET, RES, W32>(p, grid_ctas, s);
+        }
     }
     if (nv <= 32) return launch_large_p<16, 2, 16, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 64) return launch_large_p<32, 2, 8, DET, RES, W32>(p, grid_ctas, s);
