@@ -147,9 +147,20 @@ struct StagedCfg {
     int32_t n_stages;
     int32_t stage_bytes;   // one stage, all tensors
     int32_t tensor_bytes;  // one tensor's rows inside a stage
-    int32_t xch_offset;    // FP64 [nvec*8] running sum of a chunk's blocks
+    int32_t xch_offset;    // FP64 exchange of a chunk's blocks: [xch_rows][nvec*8]
+    int32_t xch_rows;      // L: every block its own row, one barrier (short blocks);
+                           // 1: a running sum in block order (64-row blocks, frees a stage)
     int32_t stage_offset;
 };
+
+// Rows of the deterministic chunk exchange: one row per block for blocks shorter than 64 rows
+// (a chunk there is only a few tiles, and one barrier per block would dominate: [1024,24,256]
+// 31.2 vs 25.1 us), a single running-sum row for 64-row blocks (the smaller exchange leaves
+// room for one more pipeline stage: H 512 x 131072 93 vs 101 us, H 1536 x 65537 124 vs 134 us).
+inline int det_xch_rows(bool det, int L, int block_rows) {
+    if (!det || L == 1) return 0;
+    return block_rows < 64 ? L : 1;
+}
 
 template <int ST, int VPT, int L, int P, bool DET, int NV, bool RES, bool W32>
 __global__ void __launch_bounds__(32 + ST * L, 1)
@@ -174,7 +185,7 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 16 * kMaxStages);
     volatile unsigned* last_flag = reinterpret_cast<volatile unsigned*>(smem + 16 * kMaxStages + 4);
     float* red = reinterpret_cast<float*>(smem + 16 * kMaxStages + 16);  // [L][2][P][SW]
-    double* xch = reinterpret_cast<double*>(smem + sc.xch_offset);       // [nvec*8] running chunk sum
+    double* xch = reinterpret_cast<double*>(smem + sc.xch_offset);       // [xch_rows][nvec*8]
     unsigned char* stages = smem + sc.stage_offset;
 
     const int NS = sc.n_stages;
@@ -511,6 +522,29 @@ __global__ void __launch_bounds__(32 + ST * L, 1)
                         *reinterpret_cast<double2*>(dst + 2 * kk) = t2;
                     }
                 }
+            } else if (sc.xch_rows > 1) {
+                // every block to its own FP64 row, one consumer barrier, then each column's
+                // blocks folded left to right
+                if (slot < nb) {
+#pragma unroll
+                    for (int i = 0; i < VPT; ++i) {
+                        const int v = ts + ST * i;
+                        if (!NV && v >= nvec) continue;
+                        double* mine = xch + (size_t)slot * nvec * 8 + 8 * v;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            mine[2 * kk] = -((double)s2[i][kk].x + (double)c2[i][kk].x);
+                            mine[2 * kk + 1] = -((double)s2[i][kk].y + (double)c2[i][kk].y);
+                        }
+                    }
+                }
+                named_bar(kAllConsumers, NCT);
+                for (int col = ctid; col < H; col += NCT) {
+                    double a = xch[col];
+                    for (int b = 1; b < nb; ++b) a += xch[(size_t)b * nvec * 8 + col];
+                    p.part[(size_t)k * H + col] = a;
+                }
+                named_bar(kAllConsumers, NCT);
             } else {
                 // the chunk's blocks folded left to right through one FP64 row: slot b adds
                 // its block to the running sum after slot b - 1 has (one consumer barrier per
@@ -1029,7 +1063,8 @@ cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     constexpr int NTEN = RES ? 3 : 2;
     constexpr size_t kBudget = 220 * 1024;
     StagedCfg sc;
-    const size_t xch = (DET && L > 1) ? (size_t)p.nvec * 8 * sizeof(double) : 0;
+    sc.xch_rows = det_xch_rows(DET, L, p.block_rows);
+    const size_t xch = (size_t)sc.xch_rows * p.nvec * 8 * sizeof(double);
     sc.xch_offset = kStagedHeader;
     sc.stage_offset = (int32_t)(kStagedHeader + ((xch + 127) & ~size_t(127)));
     sc.tensor_bytes = L * P * p.H * 2;
@@ -1128,7 +1163,7 @@ cudaError_t launch_large_nv(const BwdParams& p, int grid_ctas, cudaStream_t s) {
 template <int ST, int VPT, int L, bool DET, bool RES, bool W32>
 cudaError_t launch_large_p(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     constexpr size_t kRoom = 220 * 1024 - kStagedHeader;
-    const size_t xch = (DET && L > 1) ? (size_t)p.nvec * 8 * sizeof(double) : 0;
+    const size_t xch = (size_t)det_xch_rows(DET, L, p.block_rows) * p.nvec * 8 * sizeof(double);
     const size_t row = (size_t)(RES ? 3 : 2) * L * p.H * 2;
     if (2 * 4 * row + xch + 128 <= kRoom)
         return launch_large_nv<ST, VPT, L, 4, DET, RES, W32>(p, grid_ctas, s);
