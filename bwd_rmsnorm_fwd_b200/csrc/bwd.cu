@@ -162,8 +162,8 @@ inline int det_xch_rows(bool det, int L, int block_rows) {
     return block_rows < 64 ? L : 1;
 }
 
-template <int ST, int VPT, int L, int P, bool DET, int NV, bool RES, bool W32>
-__global__ void __launch_bounds__(32 + ST * L, 1)
+template <int ST, int VPT, int L, int P, bool DET, int NV, bool RES, bool W32, int MINB>
+__global__ void __launch_bounds__(32 + ST * L, MINB)
     bwd_staged_kernel(const BwdParams p, const StagedCfg sc, const __grid_constant__ RowMaps tm) {
     // NV != 0: the width is exactly NV vectors, every consumer thread owns VPT of them, and
     // the row size is a compile-time constant (no per-vector range checks, constant offsets)
@@ -1056,12 +1056,16 @@ namespace {
 
 cudaError_t launch_fold(const BwdParams& p, cudaStream_t s);
 
-template <int ST, int VPT, int L, int P, bool DET, int NV, bool RES, bool W32>
+// Shared memory one CTA of the staged kernel may take when MINB of them share an SM (228 KB
+// per SM, 1 KB of it reserved per CTA).
+constexpr size_t staged_budget(int minb) { return minb == 1 ? 220 * 1024 : 112 * 1024; }
+
+template <int ST, int VPT, int L, int P, bool DET, int NV, bool RES, bool W32, int MINB>
 cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
-    auto kern = bwd_staged_kernel<ST, VPT, L, P, DET, NV, RES, W32>;
+    auto kern = bwd_staged_kernel<ST, VPT, L, P, DET, NV, RES, W32, MINB>;
     constexpr int NT = 32 + ST * L;
     constexpr int NTEN = RES ? 3 : 2;
-    constexpr size_t kBudget = 220 * 1024;
+    constexpr size_t kBudget = staged_budget(MINB);
     StagedCfg sc;
     sc.xch_rows = det_xch_rows(DET, L, p.block_rows);
     const size_t xch = (size_t)sc.xch_rows * p.nvec * 8 * sizeof(double);
@@ -1081,7 +1085,7 @@ cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     if (ge != cudaSuccess) return ge;
     int grid = grid_ctas;
     if (grid <= 0) {
-        const int64_t cap = device_sm_count();
+        const int64_t cap = (int64_t)device_sm_count() * MINB;
         int64_t need = DET ? p.n_chunks : ((int64_t)p.R + L * 8 - 1) / (L * 8);
         if (need < 1) need = 1;
         grid = (int)(need < cap ? need : cap);
@@ -1151,23 +1155,24 @@ cudaError_t launch_fold(const BwdParams& p, cudaStream_t s) {
 // ST*VPT vectors and a slot has at least two warps (measured 4-16 % faster at H 1536-6144;
 // with fewer threads per row the compiler hoists a whole tile's loads once the offsets are
 // constant, and spills; the blocked-FP32 consumer measured slower with it).
-template <int ST, int VPT, int L, int P, bool DET, bool RES, bool W32>
+template <int ST, int VPT, int L, int P, bool DET, bool RES, bool W32, int MINB>
 cudaError_t launch_large_nv(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     if constexpr (DET && ST >= 64) {
         if (p.nvec == ST * VPT)
-            return launch_large<ST, VPT, L, P, DET, ST * VPT, RES, W32>(p, grid_ctas, s);
+            return launch_large<ST, VPT, L, P, DET, ST * VPT, RES, W32, MINB>(p, grid_ctas, s);
     }
-    return launch_large<ST, VPT, L, P, DET, 0, RES, W32>(p, grid_ctas, s);
+    return launch_large<ST, VPT, L, P, DET, 0, RES, W32, MINB>(p, grid_ctas, s);
 }
 
-template <int ST, int VPT, int L, bool DET, bool RES, bool W32>
+// MINB: CTAs of the layout that share an SM (each with its own producer and stage ring).
+template <int ST, int VPT, int L, bool DET, bool RES, bool W32, int MINB = 1>
 cudaError_t launch_large_p(const BwdParams& p, int grid_ctas, cudaStream_t s) {
-    constexpr size_t kRoom = 220 * 1024 - kStagedHeader;
+    constexpr size_t kRoom = staged_budget(MINB) - kStagedHeader;
     const size_t xch = (size_t)det_xch_rows(DET, L, p.block_rows) * p.nvec * 8 * sizeof(double);
     const size_t row = (size_t)(RES ? 3 : 2) * L * p.H * 2;
     if (2 * 4 * row + xch + 128 <= kRoom)
-        return launch_large_nv<ST, VPT, L, 4, DET, RES, W32>(p, grid_ctas, s);
-    return launch_large_nv<ST, VPT, L, 2, DET, RES, W32>(p, grid_ctas, s);
+        return launch_large_nv<ST, VPT, L, 4, DET, RES, W32, MINB>(p, grid_ctas, s);
+    return launch_large_nv<ST, VPT, L, 2, DET, RES, W32, MINB>(p, grid_ctas, s);
 }
 
 // Slot layout per width: ST threads per slot, VPT vectors per thread, L slots per CTA.  L is
@@ -1196,8 +1201,18 @@ cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     if (nv <= 32) return launch_large_p<16, 2, 16, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 64) return launch_large_p<32, 2, 8, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 128) return launch_large_p<64, 2, 4, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 192) return launch_large_p<96, 2, 4, DET, RES, W32>(p, grid_ctas, s);
-    if (nv <= 256) return launch_large_p<256, 1, 2, DET, RES, W32>(p, grid_ctas, s);
+    if constexpr (DET) {
+        // H 2048: one slot per CTA, two CTAs per SM, each with its own producer and ring, so
+        // neither slot waits for the other to release a stage (the order's L is 1 at this
+        // width).  Measured: H 2048 x 8192 30.9 vs 34.2 us, level at 65537 rows; the same at
+        // H 1536 (192 x 1) was much slower (168 vs 122 us), so H 1536 keeps 96 x 2 x 4.
+        if (nv <= 192) return launch_large_p<96, 2, 4, DET, RES, W32>(p, grid_ctas, s);
+        if (nv <= 256) return launch_large_p<256, 1, 1, DET, RES, W32, 2>(p, grid_ctas, s);
+    }
+    // blocked FP32 (measured: H 1536 x 65537 112 vs 116 us with 192 x 1 against 96 x 2; H 2048
+    // x 65537 143 vs 155 us with 128 x 2 against 256 x 1)
+    if (nv <= 192) return launch_large_p<192, 1, 2, DET, RES, W32>(p, grid_ctas, s);
+    if (nv <= 256) return launch_large_p<128, 2, 2, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 384) return launch_large_p<128, 3, 2, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 512) return launch_large_p<512, 1, 1, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 640) return launch_large_p<640, 1, 1, DET, RES, W32>(p, grid_ctas, s);
@@ -1247,6 +1262,7 @@ int bwd_slots_for_width(int H) {
     if (nv <= 32) return 16;
     if (nv <= 64) return 8;
     if (nv <= 192) return 4;
+    if (nv <= 256) return 1;
     if (nv <= 384) return 2;
     return 1;
 }
