@@ -1189,16 +1189,17 @@ cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
         if (nv <= 64 && (int64_t)p.R * p.H < kWarpBwdMaxElems)
             return dispatch_warp_bwd<RES, W32>(p, grid_ctas, s);
     }
+    // H <= 256, both modes: half-warp slots, 8 per CTA, two CTAs per SM, each with its own
+    // producer and ring (measured against one CTA of 16 slots: deterministic [1024,24,256]
+    // 21.0 vs 24.5 us, [16384,4,256] 34.3 vs 38.5 us; blocked FP32 H 256 x 1M 278 vs 295 us;
+    // within 2 % either way at [16384,24,256]; slower at H 512, which keeps one CTA)
+    if (nv <= 32) return launch_large_p<16, 2, 8, DET, RES, W32, 2>(p, grid_ctas, s);
     if constexpr (DET) {
-        // thinner slots for the narrowest rows at many rows: twice the consumer warps
-        // (measured: H 512 x 131072 100 vs 105 us, [16384,24,256] 156 vs 161 us; slower below:
-        // [1024,24,256] 28.9 vs 25.1 us, [16384,4,256] 39.8 vs 38.6 us); same L, same order
-        if (p.R >= kThinDetRows) {
-            if (nv <= 32) return launch_large_p<32, 1, 16, DET, RES, W32>(p, grid_ctas, s);
-            if (nv <= 64) return launch_large_p<64, 1, 8, DET, RES, W32>(p, grid_ctas, s);
-        }
+        // thinner slots at H 512 from 131072 rows: twice the consumer warps (H 512 x 131072
+        // 100 vs 105 us; slower at fewer rows); same L, same order
+        if (p.R >= kThinDetRows && nv <= 64)
+            return launch_large_p<64, 1, 8, DET, RES, W32>(p, grid_ctas, s);
     }
-    if (nv <= 32) return launch_large_p<16, 2, 16, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 64) return launch_large_p<32, 2, 8, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 128) return launch_large_p<64, 2, 4, DET, RES, W32>(p, grid_ctas, s);
     if constexpr (DET) {
@@ -1259,7 +1260,7 @@ cudaError_t dispatch_small(const BwdParams& p, cudaStream_t s) {
 
 int bwd_slots_for_width(int H) {
     const int nv = H / 8;
-    if (nv <= 32) return 16;
+    if (nv <= 32) return 8;
     if (nv <= 64) return 8;
     if (nv <= 192) return 4;
     if (nv <= 256) return 1;

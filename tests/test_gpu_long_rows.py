@@ -1,7 +1,7 @@
 """The very long narrow-row regime: H 256 rows at T 1,048,576 (the pages' H256 T1048576 rows,
 BF16 and FP32 weight), both backward modes.  Row outputs are checked on sampled rows the
 oracle computes one by one, dw over every row; the deterministic bits across three grids
-(the order's 64-row blocks in 1024 chunks at this size); and the blocked-FP32 program's
+(the order's 64-row blocks in 2048 chunks at this size); and the blocked-FP32 program's
 cut-over at 2^24 elements from both sides, against the full oracle."""
 
 from __future__ import annotations
@@ -28,7 +28,7 @@ def sample_idx(R, n=512, seed=1):
 def test_h256_million_rows(wdt):
     T, H = 1 << 20, 256
     B, L, S = api.det_plan(T, 1, H)
-    assert (B, L, S) == (64, 16, 16)            # 1024 chunks of 1024 rows
+    assert (B, L, S) == (64, 8, 16)             # 2048 chunks of 512 rows
     x = synth.rows(80, "x", T, H)
     dy = synth.rows(80, "dy", T, H)
     w = synth.weight(80, H, wdt)
