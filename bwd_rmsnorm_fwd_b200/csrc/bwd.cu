@@ -140,6 +140,35 @@ __device__ __forceinline__ void slot_dots(const float (&v)[P], float (&dot)[P], 
 // then waits for its copies in flight before the CTA exits.
 // ============================================================================================
 
+// Blocked-FP32 finish, run by the last CTA to take a ticket: the FP64 column totals become dw
+// and are cleared for the next call.  The loads go out in batches: the stores to dw and to
+// the totals may alias later loads as far as the compiler knows, so a plain per-column loop
+// would wait one L2 round trip per column (24 in a row at H 6144 with 256 threads).
+constexpr int kFinishBatch = 8;
+
+__device__ __forceinline__ void finish_dw(const BwdParams& p, int tid, int nt) {
+    const int H = p.H;
+    for (int c0 = tid; c0 < H; c0 += kFinishBatch * nt) {
+        double tot[kFinishBatch];
+        float prev[kFinishBatch];
+#pragma unroll
+        for (int u = 0; u < kFinishBatch; ++u) {
+            const int c = c0 + u * nt;
+            tot[u] = c < H ? __ldcg(p.acc + c) : 0.0;
+            prev[u] = (p.accumulate && c < H) ? __ldcg(p.dw + c) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kFinishBatch; ++u) {
+            const int c = c0 + u * nt;
+            if (c < H) {
+                const float v = __double2float_rn(tot[u]);
+                p.dw[c] = p.accumulate ? __fadd_rn(prev[u], v) : v;
+                p.acc[c] = 0.0;
+            }
+        }
+    }
+}
+
 constexpr int kMaxStages = 16;
 constexpr int kStagedHeader = 2048;  // barriers, flags, slot reduction buffers
 
@@ -608,10 +637,7 @@ __global__ void __launch_bounds__(32 + ST * L, MINB)
         named_bar(kAllConsumers, NCT);
         if (*last_flag) {
             __threadfence();
-            for (int col = ctid; col < H; col += NCT) {
-                store_dw(p, col, __ldcg(p.acc + col));
-                p.acc[col] = 0.0;
-            }
+            finish_dw(p, ctid, NCT);
             if (ctid == 0) *p.ticket = 0u;
         }
     }
@@ -807,10 +833,7 @@ __global__ void __launch_bounds__(32 * kWarpBwdWarps) bwd_warp_kernel(const BwdP
     __syncthreads();
     if (last) {
         __threadfence();
-        for (int col = threadIdx.x; col < H; col += blockDim.x) {
-            store_dw(p, col, __ldcg(p.acc + col));
-            p.acc[col] = 0.0;
-        }
+        finish_dw(p, threadIdx.x, blockDim.x);
         if (threadIdx.x == 0) *p.ticket = 0u;
     }
 }
