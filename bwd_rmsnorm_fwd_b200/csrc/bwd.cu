@@ -1081,7 +1081,9 @@ cudaError_t launch_fold(const BwdParams& p, cudaStream_t s);
 
 // Shared memory one CTA of the staged kernel may take when MINB of them share an SM (228 KB
 // per SM, 1 KB of it reserved per CTA).
-constexpr size_t staged_budget(int minb) { return minb == 1 ? 220 * 1024 : 112 * 1024; }
+constexpr size_t staged_budget(int minb) {
+    return minb == 1 ? 220 * 1024 : minb == 2 ? 112 * 1024 : minb == 3 ? 74 * 1024 : 55 * 1024;
+}
 
 template <int ST, int VPT, int L, int P, bool DET, int NV, bool RES, bool W32, int MINB>
 cudaError_t launch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
@@ -1215,7 +1217,13 @@ cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     // H <= 256, both modes: half-warp slots, 8 per CTA, two CTAs per SM, each with its own
     // producer and ring (measured against one CTA of 16 slots: deterministic [1024,24,256]
     // 21.0 vs 24.5 us, [16384,4,256] 34.3 vs 38.5 us; blocked FP32 H 256 x 1M 278 vs 295 us;
-    // within 2 % either way at [16384,24,256]; slower at H 512, which keeps one CTA)
+    // within 2 % either way at [16384,24,256]; slower at H 512, which keeps one CTA).  The
+    // deterministic mode takes three CTAs per SM from 131072 rows (128 registers, no spill:
+    // [16384,24,256] 136 vs 154 us, H 256 x 1M 319 vs 343 us; 4 % slower at 65536 rows)
+    if constexpr (DET) {
+        if (nv <= 32 && p.R >= kThinDetRows)
+            return launch_large_p<16, 2, 8, DET, RES, W32, 3>(p, grid_ctas, s);
+    }
     if (nv <= 32) return launch_large_p<16, 2, 8, DET, RES, W32, 2>(p, grid_ctas, s);
     if constexpr (DET) {
         // thinner slots at H 512 from 131072 rows: twice the consumer warps (H 512 x 131072
@@ -1226,12 +1234,14 @@ cudaError_t dispatch_large(const BwdParams& p, int grid_ctas, cudaStream_t s) {
     if (nv <= 64) return launch_large_p<32, 2, 8, DET, RES, W32>(p, grid_ctas, s);
     if (nv <= 128) return launch_large_p<64, 2, 4, DET, RES, W32>(p, grid_ctas, s);
     if constexpr (DET) {
-        // H 2048: one slot per CTA, two CTAs per SM, each with its own producer and ring, so
-        // neither slot waits for the other to release a stage (the order's L is 1 at this
-        // width).  Measured: H 2048 x 8192 30.9 vs 34.2 us, level at 65537 rows; the same at
-        // H 1536 (192 x 1) was much slower (168 vs 122 us), so H 1536 keeps 96 x 2 x 4.
+        // H 2048: one slot of 128 threads with two vectors each per CTA, three CTAs per SM,
+        // each with its own producer and ring, so no slot waits for another to release a
+        // stage (the order's L is 1 at this width; 128 registers).  Measured at 65537 rows:
+        // 157 us against 178 with 256 x 1 at two CTAs per SM; at four CTAs per SM the
+        // registers spill.  At H 1536 (L 4) neither 64 x 3 x 4 (spills at two CTAs per SM,
+        // slower at one) nor 192 x 1 at two CTAs per SM beats 96 x 2 x 4.
         if (nv <= 192) return launch_large_p<96, 2, 4, DET, RES, W32>(p, grid_ctas, s);
-        if (nv <= 256) return launch_large_p<256, 1, 1, DET, RES, W32, 2>(p, grid_ctas, s);
+        if (nv <= 256) return launch_large_p<128, 2, 1, DET, RES, W32, 3>(p, grid_ctas, s);
     }
     // blocked FP32 (measured: H 1536 x 65537 112 vs 116 us with 192 x 1 against 96 x 2; H 2048
     // x 65537 143 vs 155 us with 128 x 2 against 256 x 1)
