@@ -267,6 +267,66 @@ def make_inputs(T, H, wdt, seed, device, torch):
     return x, dy, w
 
 
+HEAD_VIEWS = {"24x256_pages": (24, 12288, 512), "24x256_dense": (24, 6144, 256),
+              "4x256": (4, 1024, 256)}
+
+
+def head_view_inputs(T, view, device, torch):
+    """x, dy as a per-head view [T, heads, 256] of one allocation each (the pages' strided
+    layout, a dense one, or four heads), and an FP32 weight of 256."""
+    heads, st, sk = HEAD_VIEWS[view]
+    n = (T - 1) * st + (heads - 1) * sk + 256
+    g = torch.Generator(device=device)
+    g.manual_seed(5)
+    bx = torch.randn(n, generator=g, device=device).to(torch.bfloat16)
+    bd = torch.randn(n, generator=g, device=device).to(torch.bfloat16)
+    x = torch.as_strided(bx, (T, heads, 256), (st, sk, 1))
+    dy = torch.as_strided(bd, (T, heads, 256), (st, sk, 1))
+    w = 1 + 0.1 * torch.randn(256, generator=g, device=device)
+    return x, dy, w
+
+
+def profile_case(spec, torch, api, dev, calls=3):
+    """Runs one library call of one configuration `calls` times with L2 flushed before each
+    (the program a profiler capture runs).  spec = OP:H:T[:FORM[:W]]: OP fwd, bwd_det or
+    bwd_nondet; FORM plain (default), res (H 6144 residual rows) or a per-head view
+    (24x256_pages, 24x256_dense, 4x256; H is 256 there and T counts tokens); W bf16
+    (default) or fp32."""
+    parts = spec.split(":")
+    op, H, T = parts[0], int(parts[1]), int(parts[2])
+    form = parts[3] if len(parts) > 3 else "plain"
+    wdt = parts[4] if len(parts) > 4 else "bf16"
+    if op not in ("fwd", "bwd_det", "bwd_nondet"):
+        raise SystemExit(f"unknown op {op!r}")
+    res = dh = None
+    if form in HEAD_VIEWS:
+        x, dy, w = head_view_inputs(T, form, dev, torch)
+    else:
+        x, dy, w = make_inputs(T, H, wdt, 6, dev, torch)
+        if form == "res":
+            res, dh, _ = make_inputs(T, H, "bf16", 4, dev, torch)
+        elif form != "plain":
+            raise SystemExit(f"unknown form {form!r}")
+    if res is not None:
+        h, _, rstd = api.rmsnorm_train_fwd(x, w, residual=res)
+    else:
+        h = x
+        _, rstd = api.rmsnorm_train_fwd(x, w)
+    ws = api.Workspace(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)  # > L2
+    for _ in range(calls):
+        flush.zero_()
+        if op == "fwd":
+            api.rmsnorm_train_fwd(x, w, residual=res)
+        else:
+            api.rmsnorm_train_bwd(h, w, rstd, dy, deterministic=op == "bwd_det", dh=dh,
+                                  workspace=ws)
+    if dev.type == "cuda":
+        torch.cuda.synchronize(dev)
+    api.status(ws)
+    print("profile case done:", spec)
+
+
 def call_spans_us(events, flush_tag="FillFunctor"):
     """Per-call spans from device records (name, start_us, end_us) of a loop that flushes L2
     before every call: records sorted by start, cut at every flush kernel; a call's span runs
@@ -446,20 +506,13 @@ def sweep(torch, api, flush, peak, dev, groups=SWEEP_GROUPS, rounds=3, reps=67):
         run_group(e)
         del e, x, dy, res, dh
     for T in (1024, 16384) if "per-head" in groups else ():
-        for name, heads, st, sk in (("24x256_pages", 24, 12288, 512),
-                                    ("24x256_dense", 24, 6144, 256), ("4x256", 4, 1024, 256)):
+        for name in HEAD_VIEWS:
             e = []
-            n = (T - 1) * st + (heads - 1) * sk + 256
-            g = torch.Generator(device=dev)
-            g.manual_seed(5)
-            bx = torch.randn(n, generator=g, device=dev).to(torch.bfloat16)
-            bd = torch.randn(n, generator=g, device=dev).to(torch.bfloat16)
-            x = torch.as_strided(bx, (T, heads, 256), (st, sk, 1))
-            dy = torch.as_strided(bd, (T, heads, 256), (st, sk, 1))
-            w = 1 + 0.1 * torch.randn(256, generator=g, device=dev)
+            x, dy, w = head_view_inputs(T, name, dev, torch)
+            heads = HEAD_VIEWS[name][0]
             ops(e, "per-head", name, x, dy, w, 256, T, T * heads, "fp32")
             run_group(e)
-            del e, bx, bd
+            del e, x, dy
     for H in (1536, 2048, 4096, 5120, 6144) if "large-T" in groups else ():
         for wdt in ("bf16", "fp32"):
             e = []
@@ -579,6 +632,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows", type=int, default=HEAD_T, help="T of the headline step")
     ap.add_argument("--width", type=int, default=HEAD_H, help="H of the headline step")
+    ap.add_argument("--profile-case", default=None, metavar="OP:H:T[:FORM[:W]]",
+                    help="run one call of one configuration three times (L2 flushed before "
+                         "each) and exit: the program a profiler capture runs")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -593,6 +649,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.profile_case:
+        build.build()
+        return profile_case(args.profile_case, torch, api, dev)
     dist = None
     if world > 1:
         import datetime

@@ -157,3 +157,44 @@ def test_interleaved_rounds_rotate_the_order():
                      "c", "c", "a", "a", "b", "b"]
     assert len(bench.interleaved_order(list(range(10)), 3, 67)) == 10 * 201
     assert bench.quantile([1, 2, 3, 4, 5], 0.5) == 3 and bench.quantile([4.0], 0.9) == 4.0
+
+
+class _FakeApi:
+    """Records the library calls profile_case makes (CPU tensors, no library)."""
+
+    def __init__(self):
+        self.calls = []
+
+    class Workspace:
+        def __init__(self, dev):
+            pass
+
+    def rmsnorm_train_fwd(self, x, w, residual=None):
+        self.calls.append(("fwd", tuple(x.shape), residual is not None))
+        rstd = torch.ones(x.numel() // x.shape[-1])
+        return (x, x, rstd) if residual is not None else (x, rstd)
+
+    def rmsnorm_train_bwd(self, h, w, rstd, dy, deterministic, dh=None, workspace=None):
+        self.calls.append(("bwd", tuple(h.shape), deterministic, dh is not None))
+        return h, w
+
+    def status(self, ws=None):
+        pass
+
+
+@pytest.mark.parametrize("spec, want, n", [
+    ("bwd_det:256:4:24x256_pages", ("bwd", (4, 24, 256), True, False), 3),
+    ("bwd_nondet:64:5:res", ("bwd", (5, 64), False, True), 3),
+    ("fwd:64:3:plain:fp32", ("fwd", (3, 64), False), 4),  # the setup forward gives rstd
+])
+def test_profile_case_runs_the_named_call_three_times(spec, want, n):
+    api = _FakeApi()
+    bench.profile_case(spec, torch, api, torch.device("cpu"))
+    assert api.calls.count(want) == n
+
+
+def test_profile_case_rejects_unknown_op_and_form():
+    with pytest.raises(SystemExit):
+        bench.profile_case("bwd:64:3", torch, _FakeApi(), torch.device("cpu"))
+    with pytest.raises(SystemExit):
+        bench.profile_case("fwd:64:3:diag", torch, _FakeApi(), torch.device("cpu"))
