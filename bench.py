@@ -431,12 +431,15 @@ def event_time_us(fn, flush, torch, reps=20):
 SWEEP_GROUPS = ("tiny", "small-T", "residual", "per-head", "large-T", "long-256")
 
 
-def sweep(torch, api, flush, peak, dev, groups=SWEEP_GROUPS, rounds=3, reps=67):
+def sweep(torch, api, flush, peak, dev, groups=SWEEP_GROUPS, rounds=3, reps=67,
+          device_index=None):
     """Per-configuration table for every configuration of the pages' tables: us per call
     (median, p10 and p90 of the CUPTI span of a CUDA-graph replay, cold L2, rounds x reps
     replays in interleaved rounds), an A/A floor per group (the group's first call captured
     twice and timed as two programs), CUDA-event time of the replay where a call is long
-    enough, and the fraction of the measured HBM bandwidth."""
+    enough, and the fraction of the measured HBM bandwidth.  With `device_index`, the SM clock
+    (median over NVML samples while the group's spans are taken) and any clock-event reasons
+    go into the group's first row."""
     out = []
     ws = api.Workspace(dev)
 
@@ -444,7 +447,11 @@ def sweep(torch, api, flush, peak, dev, groups=SWEEP_GROUPS, rounds=3, reps=67):
         # entries: (meta, fn, nbytes, replay); the first call is also timed as its own A/A twin
         calls = [(i, e[1]) for i, e in enumerate(entries)]
         calls.append(("aa", entries[0][1]))
+        sampler = ClockSampler(device_index) if device_index is not None else None
+        if sampler:
+            sampler.start()
         spans = time_group(calls, flush, torch, rounds, reps)
+        clk = sampler.stop() if sampler else None
         m0, ma = statistics.median(spans[0]), statistics.median(spans["aa"])
         aa = abs(m0 - ma) / ((m0 + ma) / 2)
         for i, (meta, fn, nbytes, replay) in enumerate(entries):
@@ -457,6 +464,9 @@ def sweep(torch, api, flush, peak, dev, groups=SWEEP_GROUPS, rounds=3, reps=67):
                         "replays": len(spans[i])})
             if i == 0:
                 row["aa_floor"] = round(aa, 4)
+                if clk is not None:
+                    row["group_sm_mhz"] = clk.get("sm_mhz")
+                    row["group_clock_reasons"] = clk.get("reasons")
             if replay:
                 row["replay_us"] = round(event_time_us(fn, flush, torch), 2)
             out.append(row)
@@ -743,7 +753,8 @@ def main():
         del x, dy
         torch.cuda.empty_cache()
         per_cfg = sweep(torch, api, flush, peak, dev,
-                        SWEEP_GROUPS if args.sweep == "all" else (args.sweep,))
+                        SWEEP_GROUPS if args.sweep == "all" else (args.sweep,),
+                        device_index=local)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
