@@ -435,72 +435,60 @@ __global__ void __launch_bounds__(32 + ST * L, MINB)
                                                               (size_t)(slot * P) * row_bytes);
             const uint4* sdh = reinterpret_cast<const uint4*>(sb + 2 * sc.tensor_bytes +
                                                               (size_t)(slot * P) * row_bytes);
-            // pass 1: per-thread partial sums of g * x, scaled by -rstd once per row to give
-            // the partial sums of g * (-xh) (one packed multiply per pair fewer than forming
-            // -xh here; the dot only enters dx)
-            float dpart[P], dot[P];
+            if constexpr (DET && ST <= 32) {
+                // deterministic slots within one warp: one row at a time.  Each 16-byte vector
+                // is unpacked once and kept in registers through both passes, and the row's
+                // dot is one tree over the slot's lanes (every lane takes part in every row's
+                // shuffles; rows past the slot's end are skipped after them).  Measured against
+                // the two passes below: H 256 x 1M 303 vs 319 us, H 512 x 65536 56.6 vs 59.7
+                // us, [16384,4,256] 31.3 vs 33.6 us, [1024,24,256] 20.0 vs 21.3 us; same dw
+                // bits.  The blocked-FP32 consumer measured 1-2 % slower this way and keeps the
+                // two passes.
 #pragma unroll
-            for (int q = 0; q < P; ++q) {
-                float2 d2 = make_float2(0.f, 0.f);
+                for (int q = 0; q < P; ++q) {
+                    float2 xf[VPT][4], df[VPT][4];
+                    float2 d2 = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int i = 0; i < VPT; ++i) {
-                    const int v = ts + ST * i;
-                    if (NV || v < nvec) {
-                        const uint4 xr = sx[q * nvec + v];
-                        const uint4 dr = sdy[q * nvec + v];
+                    for (int i = 0; i < VPT; ++i) {
+                        const int v = ts + ST * i;
+                        const bool in = NV || v < nvec;
+                        const uint4 xr = in ? sx[q * nvec + v] : make_uint4(0u, 0u, 0u, 0u);
+                        const uint4 dr = in ? sdy[q * nvec + v] : make_uint4(0u, 0u, 0u, 0u);
                         const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
                         const uint32_t dw4[4] = {dr.x, dr.y, dr.z, dr.w};
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            d2 = fma2(mul2(bf16x2_to_f2(dw4[k]), w2[i][k]), bf16x2_to_f2(xw[k]), d2);
+                        for (int k = 0; k < 4; ++k) {
+                            xf[i][k] = bf16x2_to_f2(xw[k]);
+                            df[i][k] = bf16x2_to_f2(dw4[k]);
+                            d2 = fma2(mul2(df[i][k], w2[i][k]), xf[i][k], d2);
+                        }
                     }
-                }
-                dpart[q] = (d2.x + d2.y) * -rs[q];
-            }
-            // the blocked-FP32 consumer of one multi-warp slot per CTA reduces row by row
-            // (measured faster there: H 4096-6144); every other layout takes the multi-row
-            // butterfly (H 2048 blocked FP32 with two slots: 137 vs 162 us)
-            if constexpr (DET || SW == 1 || L > 1)
-                slot_dots<ST, P>(dpart, dot, red, slot, buf, lane, wis);
-            else
-                slot_dots_rowwise<ST, P>(dpart, dot, red, slot, buf, lane, wis);
-            if constexpr (SW > 1) buf ^= 1;
-            // pass 2: dx = rstd (g - xh c) = rstd (g + nx c), c = -dot / H; dw, rows in order
+                    const float dotq = group_sum<ST>((d2.x + d2.y) * -rs[q]);
+                    if (base + t * P + q >= endr) continue;
+                    const float cr = -dotq * invH;
+                    const float2 c2v = make_float2(cr, cr);
+                    const float2 rs2 = make_float2(rs[q], rs[q]);
+                    const float2 nrs = make_float2(-rs[q], -rs[q]);
+                    const int row = base + t * P + q;
+                    uint16_t* dxrow = p.dx.ptr + row_offset(row, p.heads, p.dx.st, p.dx.sk);
 #pragma unroll
-            for (int q = 0; q < P; ++q) {
-                if (base + t * P + q >= endr) continue;
-                const float cr = -dot[q] * invH;
-                const float2 c2v = make_float2(cr, cr);
-                const float2 rs2 = make_float2(rs[q], rs[q]);
-                const float2 nrs = make_float2(-rs[q], -rs[q]);
-                const int row = base + t * P + q;
-                uint16_t* dxrow = p.dx.ptr + row_offset(row, p.heads, p.dx.st, p.dx.sk);
+                    for (int i = 0; i < VPT; ++i) {
+                        const int v = ts + ST * i;
+                        if (!NV && v >= nvec) continue;
+                        uint32_t hw[4] = {0u, 0u, 0u, 0u};
+                        if constexpr (RES) {
+                            const uint4 hr = sdh[q * nvec + v];
+                            hw[0] = hr.x; hw[1] = hr.y; hw[2] = hr.z; hw[3] = hr.w;
+                        }
+                        uint32_t out[4];
 #pragma unroll
-                for (int i = 0; i < VPT; ++i) {
-                    const int v = ts + ST * i;
-                    if (!NV && v >= nvec) continue;
-                    const uint4 xr = sx[q * nvec + v];
-                    const uint4 dr = sdy[q * nvec + v];
-                    const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
-                    const uint32_t dw4[4] = {dr.x, dr.y, dr.z, dr.w};
-                    uint32_t hw[4] = {0u, 0u, 0u, 0u};
-                    if constexpr (RES) {
-                        const uint4 hr = sdh[q * nvec + v];
-                        hw[0] = hr.x; hw[1] = hr.y; hw[2] = hr.z; hw[3] = hr.w;
-                    }
-                    uint32_t out[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float2 d = bf16x2_to_f2(dw4[k]);
-                        const float2 nx = mul2(bf16x2_to_f2(xw[k]), nrs);
-                        const float2 g = mul2(d, w2[i][k]);
-                        float2 o = mul2(fma2(nx, c2v, g), rs2);
-                        if constexpr (RES) o = add2(o, bf16x2_to_f2(hw[k]));
-                        out[k] = pack2(o);
-                        if constexpr (DET) {
-                            // -p and its exact error -e = fma(d, -xh, p) (two scalar FMAs with
-                            // a negated addend: cheaper than a packed negation), then TwoSum;
-                            // err + (-e) rounds exactly as err - e
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 d = df[i][k];
+                            const float2 nx = mul2(xf[i][k], nrs);
+                            const float2 g = mul2(d, w2[i][k]);
+                            float2 o = mul2(fma2(nx, c2v, g), rs2);
+                            if constexpr (RES) o = add2(o, bf16x2_to_f2(hw[k]));
+                            out[k] = pack2(o);
                             const float2 np = mul2(d, nx);
                             const float2 ne = make_float2(__fmaf_rn(d.x, nx.x, -np.x),
                                                           __fmaf_rn(d.y, nx.y, -np.y));
@@ -509,11 +497,92 @@ __global__ void __launch_bounds__(32 + ST * L, MINB)
                             const float2 err = add2(sub2(s2[i][k], sub2(tt, z)), sub2(np, z));
                             c2[i][k] = add2(c2[i][k], add2(err, ne));
                             s2[i][k] = tt;
-                        } else {
-                            s2[i][k] = fma2(d, nx, s2[i][k]);
+                        }
+                        st16(dxrow + 8 * v, make_uint4(out[0], out[1], out[2], out[3]));
+                    }
+                }
+            } else {
+                // pass 1: per-thread partial sums of g * x, scaled by -rstd once per row to give
+                // the partial sums of g * (-xh) (one packed multiply per pair fewer than forming
+                // -xh here; the dot only enters dx)
+                float dpart[P], dot[P];
+#pragma unroll
+                for (int q = 0; q < P; ++q) {
+                    float2 d2 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int i = 0; i < VPT; ++i) {
+                        const int v = ts + ST * i;
+                        if (NV || v < nvec) {
+                            const uint4 xr = sx[q * nvec + v];
+                            const uint4 dr = sdy[q * nvec + v];
+                            const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+                            const uint32_t dw4[4] = {dr.x, dr.y, dr.z, dr.w};
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                d2 = fma2(mul2(bf16x2_to_f2(dw4[k]), w2[i][k]),
+                                          bf16x2_to_f2(xw[k]), d2);
                         }
                     }
-                    st16(dxrow + 8 * v, make_uint4(out[0], out[1], out[2], out[3]));
+                    dpart[q] = (d2.x + d2.y) * -rs[q];
+                }
+                // the blocked-FP32 consumer of one multi-warp slot per CTA reduces row by row
+                // (measured faster there: H 4096-6144); every other layout takes the multi-row
+                // butterfly (H 2048 blocked FP32 with two slots: 137 vs 162 us)
+                if constexpr (DET || SW == 1 || L > 1)
+                    slot_dots<ST, P>(dpart, dot, red, slot, buf, lane, wis);
+                else
+                    slot_dots_rowwise<ST, P>(dpart, dot, red, slot, buf, lane, wis);
+                if constexpr (SW > 1) buf ^= 1;
+                // pass 2: dx = rstd (g - xh c) = rstd (g + nx c), c = -dot / H; dw, rows in order
+#pragma unroll
+                for (int q = 0; q < P; ++q) {
+                    if (base + t * P + q >= endr) continue;
+                    const float cr = -dot[q] * invH;
+                    const float2 c2v = make_float2(cr, cr);
+                    const float2 rs2 = make_float2(rs[q], rs[q]);
+                    const float2 nrs = make_float2(-rs[q], -rs[q]);
+                    const int row = base + t * P + q;
+                    uint16_t* dxrow = p.dx.ptr + row_offset(row, p.heads, p.dx.st, p.dx.sk);
+#pragma unroll
+                    for (int i = 0; i < VPT; ++i) {
+                        const int v = ts + ST * i;
+                        if (!NV && v >= nvec) continue;
+                        const uint4 xr = sx[q * nvec + v];
+                        const uint4 dr = sdy[q * nvec + v];
+                        const uint32_t xw[4] = {xr.x, xr.y, xr.z, xr.w};
+                        const uint32_t dw4[4] = {dr.x, dr.y, dr.z, dr.w};
+                        uint32_t hw[4] = {0u, 0u, 0u, 0u};
+                        if constexpr (RES) {
+                            const uint4 hr = sdh[q * nvec + v];
+                            hw[0] = hr.x; hw[1] = hr.y; hw[2] = hr.z; hw[3] = hr.w;
+                        }
+                        uint32_t out[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 d = bf16x2_to_f2(dw4[k]);
+                            const float2 nx = mul2(bf16x2_to_f2(xw[k]), nrs);
+                            const float2 g = mul2(d, w2[i][k]);
+                            float2 o = mul2(fma2(nx, c2v, g), rs2);
+                            if constexpr (RES) o = add2(o, bf16x2_to_f2(hw[k]));
+                            out[k] = pack2(o);
+                            if constexpr (DET) {
+                                // -p and its exact error -e = fma(d, -xh, p) (two scalar FMAs with
+                                // a negated addend: cheaper than a packed negation), then TwoSum;
+                                // err + (-e) rounds exactly as err - e
+                                const float2 np = mul2(d, nx);
+                                const float2 ne = make_float2(__fmaf_rn(d.x, nx.x, -np.x),
+                                                              __fmaf_rn(d.y, nx.y, -np.y));
+                                const float2 tt = add2(s2[i][k], np);
+                                const float2 z = sub2(tt, s2[i][k]);
+                                const float2 err = add2(sub2(s2[i][k], sub2(tt, z)), sub2(np, z));
+                                c2[i][k] = add2(c2[i][k], add2(err, ne));
+                                s2[i][k] = tt;
+                            } else {
+                                s2[i][k] = fma2(d, nx, s2[i][k]);
+                            }
+                        }
+                        st16(dxrow + 8 * v, make_uint4(out[0], out[1], out[2], out[3]));
+                    }
                 }
             }
             __syncwarp();
