@@ -198,3 +198,13 @@ def test_profile_case_rejects_unknown_op_and_form():
         bench.profile_case("bwd:64:3", torch, _FakeApi(), torch.device("cpu"))
     with pytest.raises(SystemExit):
         bench.profile_case("fwd:64:3:diag", torch, _FakeApi(), torch.device("cpu"))
+
+
+def test_clock_sampler_without_a_gpu_reports_nothing():
+    """No driver here: the sampler must report no clock rather than raise (the sweep records
+    its result per group)."""
+    s = bench.ClockSampler(0)
+    s.start()
+    c = s.stop()
+    if not s.ok:
+        assert c["sm_mhz"] is None and c["reasons"] == []
