@@ -65,8 +65,9 @@ __device__ __forceinline__ uint4 scale8(const uint4& x, float rstd, const void* 
 }
 
 // ---- rows of <= 4 vectors per lane: one warp per row (group) -----------------------------------
-template <int VPT, int ROWS, bool RES, bool W32>
-__global__ void __launch_bounds__(kFwdWarpThreads) fwd_warp_kernel(const FwdParams p) {
+// MINB: CTAs per SM the registers are capped for (launch bounds).
+template <int VPT, int ROWS, bool RES, bool W32, int MINB>
+__global__ void __launch_bounds__(kFwdWarpThreads, MINB) fwd_warp_kernel(const FwdParams p) {
     const int lane = threadIdx.x & 31;
     const int gwarp = (int)((blockIdx.x * kFwdWarpThreads + threadIdx.x) >> 5);
     const int nwarps = (int)((gridDim.x * kFwdWarpThreads) >> 5);
@@ -344,9 +345,9 @@ __global__ void __launch_bounds__(kFwdRowMaxThreads) fwd_row_cta_kernel(const Fw
 
 namespace {
 
-template <int VPT, int ROWS, bool RES, bool W32>
+template <int VPT, int ROWS, bool RES, bool W32, int MINB = 1>
 cudaError_t launch_warp(const FwdParams& p, cudaStream_t s) {
-    auto kern = fwd_warp_kernel<VPT, ROWS, RES, W32>;
+    auto kern = fwd_warp_kernel<VPT, ROWS, RES, W32, MINB>;
     static PerDevice<1> occ;
     cudaError_t e = cudaSuccess;
     const int o = resident_ctas(occ, current_device(), 0, kern, kFwdWarpThreads, 0, &e);
@@ -366,6 +367,18 @@ cudaError_t launch_warp_vpt(const FwdParams& p, bool res, bool w32, cudaStream_t
     const bool big = ROWS_BIG > 1 &&
                      (int64_t)p.R >= (int64_t)device_sm_count() * 64 * ROWS_BIG * 2;
     if (big) {
+        // four rows of one vector per warp: registers capped for four CTAs per SM (32 warps)
+        // with a BF16 weight (no spill: H 256 x 1M 180 vs 183 us) and for per-head views (an
+        // FP32 weight spills 16 bytes there, but [16384,24,256] runs 70.6 vs 76.5 us); plain
+        // FP32-weight rows keep three CTAs (176 vs 184 us at 1M rows)
+        if constexpr (VPT == 1 && ROWS_BIG == 4) {
+            if (!w32 || p.heads > 1) {
+                if (res) return w32 ? launch_warp<VPT, ROWS_BIG, true, true, 4>(p, s)
+                                    : launch_warp<VPT, ROWS_BIG, true, false, 4>(p, s);
+                return w32 ? launch_warp<VPT, ROWS_BIG, false, true, 4>(p, s)
+                           : launch_warp<VPT, ROWS_BIG, false, false, 4>(p, s);
+            }
+        }
         if (res) return w32 ? launch_warp<VPT, ROWS_BIG, true, true>(p, s)
                             : launch_warp<VPT, ROWS_BIG, true, false>(p, s);
         return w32 ? launch_warp<VPT, ROWS_BIG, false, true>(p, s)
