@@ -465,7 +465,11 @@ cudaError_t launch_fwd(const FwdParams& p, bool res, bool w32, cudaStream_t s) {
     if (need <= 2) return launch_warp_vpt<2, 2>(p, res, w32, s);
     if (need <= 3) return launch_warp_vpt<3, 1>(p, res, w32, s);
     if (need <= 4) return launch_warp_vpt<4, 1>(p, res, w32, s);
-    if (p.nvec <= 512) return launch_row_cta_vpt<2, 0>(p, res, w32, s);
+    // H 4096 from 32768 rows: four vectors per thread (128-thread CTAs), twice the loads in
+    // flight per thread (measured: H 4096 x 131072 FP32 w 335 vs 356 us, BF16 w 344 vs 347 us,
+    // residual x 65537 335 vs 350 us; 3-5 % slower at 16384 rows, mixed at H 3072)
+    if (p.nvec <= 384 || (p.nvec <= 512 && p.R < kFwdRingMinRows))
+        return launch_row_cta_vpt<2, 0>(p, res, w32, s);
     // The residual form reads two rows per row: there a two-row cp.async ring keeps enough
     // bytes in flight to pay for itself once every CTA walks many rows (measured: H 6144 x
     // 65537 rows 513 vs 529 us); for one input row it costs more than it brings.
